@@ -1,0 +1,203 @@
+"""CPU oracle for the guarded block-wise W8A8 linear layer (ctypes wrapper of oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by the
+CPU-baseline leg of bench.py.  The CUDA product path never imports it.  Arrays cross as
+numpy: BF16 as uint16 bit patterns, codes as int8, scales and outputs as float32.
+
+Each function states which passage of the pages it follows; see oracle.c for the
+arithmetic itself.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC",
+          "-shared", "-Wall", "-Wextra"]
+BLOCK = 128
+
+_lib = None
+
+
+def build(force=False, extra_flags=(), out=None):
+    """Compile oracle.c with gcc.  `extra_flags` and `out` exist for the mutation tests,
+    which build deliberately broken copies elsewhere."""
+    out = out or _LIB
+    if not force and out == _LIB and os.path.exists(out) and \
+            os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return out
+    cmd = ["gcc", *CFLAGS, *extra_flags, _SRC, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _i64(v):
+    return ctypes.c_int64(int(v))
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else ctypes.c_void_p(0)
+
+
+def load(path=None):
+    """Load (building first if needed) and return the ctypes library."""
+    global _lib
+    if path is not None:
+        lib = ctypes.CDLL(path)
+    elif _lib is not None:
+        return _lib
+    else:
+        lib = ctypes.CDLL(build())
+    for name in ["oracle_block_quantize", "oracle_block_sums", "oracle_w8a8_linear",
+                 "oracle_w8a8_linear_at", "oracle_rmsnorm", "oracle_rmsnorm_apply",
+                 "oracle_bf16_linear", "oracle_bf16_linear_at", "oracle_num_threads"]:
+        getattr(lib, name).restype = ctypes.c_int
+    lib.oracle_f32_to_bf16.restype = None
+    if path is None:
+        _lib = lib
+    return lib
+
+
+class Oracle:
+    """Bound wrapper, so that tests can run the same calls against a mutant build."""
+
+    def __init__(self, lib=None):
+        self.lib = lib or load()
+
+    # -- quantization (TurboDiffusion article, inference list items 3-4) --------------
+    def block_quantize(self, x_bits):
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        r, c = x.shape
+        q = np.empty((r, c), dtype=np.int8)
+        s = np.empty((r // BLOCK, c // BLOCK), dtype=np.float32)
+        rc = self.lib.oracle_block_quantize(_ptr(x), _i64(r), _i64(c), _ptr(q), _ptr(s))
+        if rc:
+            raise ValueError(f"block_quantize: shape {x.shape} not a multiple of 128")
+        return q, s
+
+    # -- INT32 sums per K block (TurboT2VA paper, W8A8 paragraph) ----------------------
+    def block_sums(self, xq, wq, m0=0, rows=None, n0=0, cols=None):
+        xq = np.ascontiguousarray(xq, dtype=np.int8)
+        wq = np.ascontiguousarray(wq, dtype=np.int8)
+        M, K = xq.shape
+        N = wq.shape[0]
+        rows = M - m0 if rows is None else rows
+        cols = N - n0 if cols is None else cols
+        out = np.empty((rows, cols, K // BLOCK), dtype=np.int32)
+        rc = self.lib.oracle_block_sums(_ptr(xq), _ptr(wq), _i64(M), _i64(K), _i64(N),
+                                        _i64(m0), _i64(rows), _i64(n0), _i64(cols), _ptr(out))
+        if rc:
+            raise ValueError("block_sums: bad arguments")
+        return out
+
+    # -- FP32 output of the W8A8 linear (TurboT2VA paper, W8A8 paragraph) --------------
+    def w8a8_linear(self, xq, xs, wq, ws, bias=None, m0=0, rows=None):
+        xq, xs, wq, ws, bias = _prep(xq, xs, wq, ws, bias)
+        M, K = xq.shape
+        N = wq.shape[0]
+        rows = M - m0 if rows is None else rows
+        out = np.empty((rows, N), dtype=np.float32)
+        rc = self.lib.oracle_w8a8_linear(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(bias),
+                                         _i64(M), _i64(K), _i64(N), _i64(m0), _i64(rows),
+                                         _ptr(out))
+        if rc:
+            raise ValueError("w8a8_linear: bad arguments")
+        return out
+
+    def w8a8_linear_at(self, xq, xs, wq, ws, bias, ms, ns):
+        xq, xs, wq, ws, bias = _prep(xq, xs, wq, ws, bias)
+        ms = np.ascontiguousarray(ms, dtype=np.int64)
+        ns = np.ascontiguousarray(ns, dtype=np.int64)
+        out = np.empty(ms.size, dtype=np.float32)
+        rc = self.lib.oracle_w8a8_linear_at(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(bias),
+                                            _i64(xq.shape[0]), _i64(xq.shape[1]),
+                                            _i64(wq.shape[0]), _ptr(ms), _ptr(ns),
+                                            _i64(ms.size), _ptr(out))
+        if rc:
+            raise ValueError("w8a8_linear_at: bad arguments")
+        return out
+
+    # -- RMSNorm (TurboDiffusion article, inference list item 5) -----------------------
+    def rmsnorm(self, x_bits, gamma_bits, eps, m0=0, rows=None):
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        g = np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+        M, K = x.shape
+        rows = M - m0 if rows is None else rows
+        y = np.empty((rows, K), dtype=np.uint16)
+        rstd = np.empty(rows, dtype=np.float32)
+        rc = self.lib.oracle_rmsnorm(_ptr(x), _ptr(g), ctypes.c_float(eps), _i64(M), _i64(K),
+                                     _i64(m0), _i64(rows), _ptr(y), _ptr(rstd))
+        if rc:
+            raise ValueError("rmsnorm: bad arguments")
+        return y, rstd
+
+    def rmsnorm_apply(self, x_bits, gamma_bits, rstd, m0=0):
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        g = np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+        r = np.ascontiguousarray(rstd, dtype=np.float32)
+        M, K = x.shape
+        y = np.empty((r.size, K), dtype=np.uint16)
+        rc = self.lib.oracle_rmsnorm_apply(_ptr(x), _ptr(g), _ptr(r), _i64(M), _i64(K),
+                                           _i64(m0), _i64(r.size), _ptr(y))
+        if rc:
+            raise ValueError("rmsnorm_apply: bad arguments")
+        return y
+
+    # -- BF16 fallback (TurboT2VA paper, guard paragraph) ------------------------------
+    def bf16_linear(self, x_bits, w_bits, bias=None, m0=0, rows=None):
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        M, K = x.shape
+        N = w.shape[0]
+        rows = M - m0 if rows is None else rows
+        out = np.empty((rows, N), dtype=np.float32)
+        rc = self.lib.oracle_bf16_linear(_ptr(x), _ptr(w), _ptr(b), _i64(M), _i64(K), _i64(N),
+                                         _i64(m0), _i64(rows), _ptr(out))
+        if rc:
+            raise ValueError("bf16_linear: bad arguments")
+        return out
+
+    def bf16_linear_at(self, x_bits, w_bits, bias, ms, ns):
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        ms = np.ascontiguousarray(ms, dtype=np.int64)
+        ns = np.ascontiguousarray(ns, dtype=np.int64)
+        out = np.empty(ms.size, dtype=np.float32)
+        rc = self.lib.oracle_bf16_linear_at(_ptr(x), _ptr(w), _ptr(b), _i64(x.shape[0]),
+                                            _i64(x.shape[1]), _i64(w.shape[0]), _ptr(ms),
+                                            _ptr(ns), _i64(ms.size), _ptr(out))
+        if rc:
+            raise ValueError("bf16_linear_at: bad arguments")
+        return out
+
+    def f32_to_bf16(self, a):
+        a = np.ascontiguousarray(a, dtype=np.float32)
+        out = np.empty(a.shape, dtype=np.uint16)
+        self.lib.oracle_f32_to_bf16(_ptr(a), _i64(a.size), _ptr(out))
+        return out
+
+    def num_threads(self):
+        return int(self.lib.oracle_num_threads())
+
+
+def _prep(xq, xs, wq, ws, bias):
+    return (np.ascontiguousarray(xq, dtype=np.int8), np.ascontiguousarray(xs, dtype=np.float32),
+            np.ascontiguousarray(wq, dtype=np.int8), np.ascontiguousarray(ws, dtype=np.float32),
+            None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16))
+
+
+_default = None
+
+
+def default():
+    """The oracle built from oracle.c as committed."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
