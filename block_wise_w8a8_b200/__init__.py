@@ -1,0 +1,234 @@
+"""Python binding of libw8a8 (the C ABI in include/w8a8.h).
+
+Argument marshalling only: every step of the W8A8 linear layer runs in the library's
+sm_100a kernels.  PyTorch provides device memory and streams.  Tensors must be CUDA,
+contiguous, and of the dtype each entry point states; BF16 is the only activation and
+weight dtype (a tensor of another dtype is rejected here, before the library is called).
+There is no CPU path: without the built library every call raises.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw8a8.so")
+
+PATH_INT8, PATH_BF16, PATH_NONE = 0, 1, 2
+DEVERR_NONE, DEVERR_TIMEOUT = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "not device memory",
+           4: "alignment", 5: "workspace", 6: "CUDA error"}
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn}: status {code} ({_STATUS.get(code, '?')})")
+        self.code = code
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("w_bf16", ctypes.c_void_p),
+                ("wq", ctypes.c_void_p), ("ws", ctypes.c_void_p)]
+
+
+_lib = None
+_SIGS = {
+    "w8a8_quantize_weight": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                             ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_quantize_act": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                          ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_rmsnorm_quantize_act": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                  ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_linear": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
+                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                    ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
+    "w8a8_linear_prequant": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                             ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p,
+                             ctypes.c_void_p],
+    "w8a8_bf16_linear": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                         ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p],
+    "w8a8_debug_block_sums": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_debug_wait_timeout": [ctypes.c_uint64, ctypes.c_void_p],
+}
+
+
+def lib():
+    """The loaded library (ctypes.CDLL).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.w8a8_linear_workspace_bytes.argtypes = [ctypes.c_int64] * 3
+        L.w8a8_linear_workspace_bytes.restype = ctypes.c_size_t
+        L.w8a8_device_error.argtypes = []
+        L.w8a8_device_error.restype = ctypes.c_int
+        L.w8a8_last_cuda_error.argtypes = []
+        L.w8a8_last_cuda_error.restype = ctypes.c_char_p
+        L.w8a8_status_string.argtypes = [ctypes.c_int]
+        L.w8a8_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(fn, code):
+    if code != 0:
+        err = W8A8Error(fn, code)
+        if code == 6:
+            err.args = (err.args[0] + ": " + lib().w8a8_last_cuda_error().decode(),)
+        raise err
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def quantize_act(x, xq=None, xs=None):
+    """Block-wise 128x128 INT8 quantization of a BF16 [M, K] matrix -> (xq int8 [M, K],
+    xs float32 [M/128, K/128])."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=x.device) if xs is None else xs
+    _check("w8a8_quantize_act", lib().w8a8_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(xs),
+                                                         _stream(x.device)))
+    return xq, xs
+
+
+def quantize_weight(w):
+    """Block-wise 128x128 INT8 quantization of a BF16 weight [N, K] -> (wq, ws)."""
+    _need(w, torch.bfloat16, "w")
+    N, K = w.shape
+    wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    ws = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device)
+    _check("w8a8_quantize_weight", lib().w8a8_quantize_weight(_ptr(w), N, K, _ptr(wq), _ptr(ws),
+                                                               _stream(w.device)))
+    return wq, ws
+
+
+def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):
+    """RMSNorm (FP64 row sums, FP32 rstd, bf16((x * rstd) * gamma)) fused with the block
+    quantizer -> (xq, xs, rstd)."""
+    _need(x, torch.bfloat16, "x")
+    _need(gamma, torch.bfloat16, "gamma")
+    M, K = x.shape
+    dev = x.device
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
+    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=dev) if xs is None else xs
+    rstd = torch.empty((M,), dtype=torch.float32, device=dev) if rstd is None else rstd
+    _check("w8a8_rmsnorm_quantize_act",
+           lib().w8a8_rmsnorm_quantize_act(_ptr(x), _ptr(gamma), float(eps), M, K, _ptr(xq),
+                                           _ptr(xs), _ptr(rstd), _stream(dev)))
+    return xq, xs, rstd
+
+
+class W8A8Weight:
+    """A linear layer's weight: the retained BF16 copy plus, when N and K are multiples of
+    128, its INT8 codes and block scales (quantized once, at construction)."""
+
+    def __init__(self, w_bf16, wq=None, ws=None):
+        _need(w_bf16, torch.bfloat16, "w")
+        self.w = w_bf16
+        self.N, self.K = w_bf16.shape
+        if wq is None and self.N % 128 == 0 and self.K % 128 == 0 and self.N and self.K:
+            wq, ws = quantize_weight(w_bf16)
+        self.wq, self.ws = wq, ws
+        self._rec = _Weight(self.N, self.K, w_bf16.data_ptr(),
+                            0 if wq is None else wq.data_ptr(),
+                            0 if ws is None else ws.data_ptr())
+
+    def record(self):
+        return ctypes.byref(self._rec)
+
+
+def linear_workspace_bytes(M, K, N):
+    return int(lib().w8a8_linear_workspace_bytes(M, K, N))
+
+
+def linear(x, weight, bias=None, out=None, workspace=None, return_path=False):
+    """The guarded W8A8 linear: y = x W^T + bias in BF16.  x: [..., K] BF16 (leading
+    dimensions flattened to M).  INT8 path when M, K, N are multiples of 128, else BF16."""
+    _need(x, torch.bfloat16, "x")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias")
+    K = x.shape[-1]
+    M = math.prod(x.shape[:-1])
+    N = weight.N
+    dev = x.device
+    out = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, device=dev) if out is None else out
+    need = linear_workspace_bytes(M, K, N)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    path = ctypes.c_int(-1)
+    _check("w8a8_linear", lib().w8a8_linear(
+        _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), ctypes.byref(path), _stream(dev)))
+    return (out, path.value) if return_path else out
+
+
+def linear_prequant(xq, xs, weight, bias=None, out=None):
+    """The INT8 block-scaled GEMM on already-quantized activations."""
+    _need(xq, torch.int8, "xq")
+    _need(xs, torch.float32, "xs")
+    M, K = xq.shape
+    out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _check("w8a8_linear_prequant", lib().w8a8_linear_prequant(
+        _ptr(xq), _ptr(xs), M, K, weight.record(), _ptr(bias), _ptr(out), _stream(xq.device)))
+    return out
+
+
+def bf16_linear(x, w, bias=None, out=None):
+    """The BF16 GEMM the guard falls back to: y = x w^T + bias, any shape."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("w8a8_bf16_linear", lib().w8a8_bf16_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(out),
+                                                       M, K, N, _stream(x.device)))
+    return out
+
+
+def debug_block_sums(xq, wq):
+    """INT32 per-K-block partial products [M, N, K/128] from the tensor-core main loop."""
+    _need(xq, torch.int8, "xq")
+    _need(wq, torch.int8, "wq")
+    M, K = xq.shape
+    N = wq.shape[0]
+    out = torch.empty((M, N, K // 128), dtype=torch.int32, device=xq.device)
+    _check("w8a8_debug_block_sums", lib().w8a8_debug_block_sums(
+        _ptr(xq), _ptr(wq), M, K, N, _ptr(out), _stream(xq.device)))
+    return out
+
+
+def debug_wait_timeout(timeout_ns, device=None):
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check("w8a8_debug_wait_timeout", lib().w8a8_debug_wait_timeout(int(timeout_ns), _stream(dev)))
+
+
+def device_error():
+    """Synchronize and return (and clear) the library's device error word."""
+    return int(lib().w8a8_device_error())

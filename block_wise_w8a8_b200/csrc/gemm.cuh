@@ -1,0 +1,548 @@
+// gemm.cuh -- persistent warp-specialised tcgen05 GEMM for sm_100a.
+//
+// Modes
+//   kI8Scaled : the block-scaled W8A8 GEMM (TurboT2VA paper, inference-stack section,
+//               W8A8 operator paragraph: the blockwise strategy applies the scales along
+//               the reduction dimension; TurboDiffusion article, inference list item 4:
+//               INT8 tensor cores).  For every 128-wide K block kb the INT32 partial
+//               product P[m,n,kb] of the INT8 codes is formed by tcgen05.mma kind::i8 in
+//               tensor memory, then the epilogue warps add float(P) * (xs * ws) into FP32
+//               running sums held in registers.  After the last block: + bias, BF16 store.
+//   kI8Dump   : same main loop; the epilogue writes P[m,n,kb] itself (test hook).
+//   kBf16     : BF16 x BF16 -> FP32 GEMM (kind::f16) for the guard's fallback (TurboT2VA
+//               paper, guard paragraph), FP32 accumulation over all of K in tensor memory.
+//
+// Tile 128 x 256 (BM x BN), one 128-byte K slice per pipeline stage (128 INT8 or 64 BF16
+// elements = exactly one K block of the INT8 path), 4 stages of 48 KB in shared memory,
+// filled by TMA with 128-byte swizzle.  Twelve warps in three warpgroups.  Warpgroup 0:
+// warp 0 is the TMA producer, warp 1 allocates TMEM and issues the MMAs (one thread),
+// warps 2-3 only wait for the end.  Warpgroups 1-2 (warps 4-11) are the epilogue; warp w
+// reads TMEM lanes 32 (w % 4) .. + 31 (the rows it may access) and columns
+// 128 ((w - 4) / 4) .. + 127.  The kernel is launched with 168 registers per thread (the
+// most 12 warps allow: each SM sub-partition holds 16K registers and 3 of the warps);
+// warpgroup 0 then gives registers back (setmaxnreg.dec to 80) and the epilogue
+// warpgroups take them (setmaxnreg.inc to 208), enough for 128 FP32 running sums per
+// thread.  128 * 80 + 256 * 208 = 63488 <= 384 * 168, the launch's total.
+// Two 256-column accumulators in TMEM (all 512 columns) let the MMA of one K block (INT8)
+// or tile (BF16) overlap the epilogue of the previous one.
+//
+// INT32 -> FP32 without conversion instructions: each INT8 accumulator is pre-filled with
+// the bit pattern of 1.5 * 2^23 (0x4B400000) and the MMAs accumulate onto it.  Because
+// |P| <= 128 * 127^2 < 2^22, the 32-bit word afterwards is the FP32 number 12582912 + P
+// exactly; one FP32 subtraction recovers float(P) exactly.  The epilogue then re-fills
+// the accumulator with the pattern for the next K block.
+#pragma once
+
+#include "common.cuh"
+
+namespace w8a8 {
+namespace gemm {
+
+enum class Mode : int { kI8Scaled = 0, kI8Dump = 1, kBf16 = 2 };
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int KSLICE_BYTES = 128;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * KSLICE_BYTES;
+constexpr int B_BYTES = BN * KSLICE_BYTES;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int EPI_WARP0 = 4;                 // first epilogue warp (warpgroup 1)
+constexpr int NUM_THREADS = 128 + NUM_EPI_WARPS * 32;
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 80;             // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsEpilogue = 208;           // warpgroups 1-2 after setmaxnreg.inc
+static_assert(128 * kRegsControl + 256 * kRegsEpilogue <= NUM_THREADS * kLaunchRegs,
+              "register split exceeds the launch's registers");
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int KB_MAX = 512;                  // K <= 65536 on the INT8 path
+constexpr uint32_t kAccInit = 0x4B400000u;   // FP32 1.5 * 2^23
+constexpr float kAccInitF = 12582912.0f;
+constexpr int TILE_GROUP = 16;               // M tiles per rasterisation group
+
+struct alignas(1024) Smem {
+    uint8_t a[STAGES][A_BYTES];
+    uint8_t b[STAGES][B_BYTES];
+    float sx[2][KB_MAX];           // [tile parity][kb]: xs[tm, kb]
+    float sw[2][2][KB_MAX];        // [tile parity][N half][kb]: ws[2 tn + half, kb]
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t mma_done;
+    uint64_t sready[2];            // scale table sprod[b] written (all epilogue threads)
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+struct Params {
+    int64_t M, N, K;
+    int32_t num_tm, num_tn, num_tiles, kslices;
+    const float *xs;          // [M/128, K/128] (INT8 modes)
+    const float *ws;          // [N/128, K/128] (INT8 modes)
+    const uint16_t *bias;     // [N] BF16 or null
+    uint16_t *y;              // [M, N] BF16
+    int32_t *dump;            // [M, N, K/128] (dump mode)
+};
+
+__device__ __forceinline__ void tile_coords(int t, int num_tm, int num_tn, int &tm, int &tn)
+{
+    const int per_group = TILE_GROUP * num_tn;
+    const int group = t / per_group;
+    const int first = group * TILE_GROUP;
+    const int gsz = min(num_tm - first, TILE_GROUP);
+    const int local = t - group * per_group;
+    tm = first + local % gsz;
+    tn = local / gsz;
+}
+
+// The block scales a tile needs, copied global -> shared with cp.async by the epilogue
+// threads one tile ahead (no registers are held while the copies are in flight):
+// sx[kb] = xs[tm, kb] and sw[h][kb] = ws[2 tn + h, kb] (0 past the last weight block).
+__device__ __forceinline__ void cp_async_4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ void scales_fetch(float *sx, float (*sw)[KB_MAX], const Params &p,
+                                             int tm, int tn, int etid, int nthreads)
+{
+    const int KB = static_cast<int>(p.K / 128);
+    const int NB = static_cast<int>(p.N / 128);
+    for (int i = etid; i < 3 * KB; i += nthreads) {
+        const int which = i / KB, kb = i - which * KB;
+        if (which == 0) {
+            cp_async_4(sx + kb, p.xs + static_cast<int64_t>(tm) * KB + kb);
+        } else {
+            const int nb = tn * 2 + which - 1;
+            if (nb < NB)
+                cp_async_4(&sw[which - 1][kb], p.ws + static_cast<int64_t>(nb) * KB + kb);
+            else
+                sw[which - 1][kb] = 0.0f;
+        }
+    }
+}
+
+template <Mode kMode>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p)
+{
+    constexpr bool kInt8 = (kMode != Mode::kBf16);
+    constexpr int kSliceElems = kInt8 ? 128 : 64;
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], NUM_EPI_WARPS);
+        }
+        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.sready[0], NUM_EPI_WARPS * 32);
+        mbar_init(&sm.sready[1], NUM_EPI_WARPS * 32);
+        sm.abort = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (warp < EPI_WARP0) {
+    regs_dec<kRegsControl>();
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+                for (int ks = 0; ks < p.kslices; ++ks, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
+                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], ks * kSliceElems, tm * BM);
+                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], ks * kSliceElems, tn * BN);
+                }
+            }
+            if (!ok) {
+                // let the copies already in flight land before shared memory is released
+                volatile int no_abort = 0;
+                const uint32_t first = it > STAGES ? it - STAGES : 0;
+                for (uint32_t j = first; j < it; ++j)
+                    mbar_wait(&sm.full[j % STAGES], (j / STAGES) & 1, &no_abort, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = kInt8 ? idesc_i8_s32(BM, BN) : idesc_bf16_f32(BM, BN);
+            uint32_t it = 0, acc_i = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                uint32_t buf = acc_i & 1;
+                if (!kInt8) {
+                    if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                for (int ks = 0; ks < p.kslices; ++ks, ++it) {
+                    const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    if (kInt8) {
+                        buf = acc_i & 1;
+                        if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!mbar_wait(&sm.full[s], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem + buf * BN;
+                    const uint64_t ad = umma_desc_sw128(smem_u32(sm.a[s]));
+                    const uint64_t bd = umma_desc_sw128(smem_u32(sm.b[s]));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        // each MMA consumes 32 bytes of K: advance start address by 32 B
+                        if (kInt8)
+                            umma_i8(d, ad + 2 * k, bd + 2 * k, idesc, 1u);
+                        else
+                            umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (ks | k) != 0);
+                    }
+                    umma_commit(&sm.empty[s]);
+                    if (kInt8) {
+                        umma_commit(&sm.tfull[buf]);
+                        ++acc_i;
+                    }
+                }
+                if (!kInt8 && ok) {
+                    umma_commit(&sm.tfull[buf]);
+                    ++acc_i;
+                }
+            }
+            // all MMAs issued by this thread complete before TMEM is released
+            umma_commit(&sm.mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(&sm.mma_done, 0, &no_abort, 100000000ull);
+        }
+    }
+    } else {
+        regs_inc<kRegsEpilogue>();
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - EPI_WARP0;
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
+        const int etid = ew * 32 + static_cast<int>(lane);
+        const int row = quarter * 32 + static_cast<int>(lane);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + half * 128;
+
+        // The accumulator re-fill pattern lives in 16 registers for the whole kernel
+        // (tcgen05.st takes its sources from consecutive registers).
+        uint32_t fill[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            fill[i] = kAccInit;
+        if (kInt8) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    tmem_st16(lane_base + b * BN + c * 16, fill);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&sm.tempty[0]);
+            mbar_arrive(&sm.tempty[1]);
+        }
+
+        uint32_t acc_i = 0;
+        if (kMode == Mode::kI8Scaled) {
+            const int KB = static_cast<int>(p.K / 128);
+            constexpr int kEpiThreads = NUM_EPI_WARPS * 32;
+            if (static_cast<int>(blockIdx.x) < p.num_tiles) {
+                int tm, tn;
+                tile_coords(blockIdx.x, p.num_tm, p.num_tn, tm, tn);
+                scales_fetch(sm.sx[0], sm.sw[0], p, tm, tn, etid, kEpiThreads);
+                cp_async_wait_all();
+            }
+            mbar_arrive(&sm.sready[0]);
+            // No named barriers here: every wait of the epilogue is a bounded mbarrier
+            // wait, so an abort can never leave part of the warps parked in bar.sync.
+            int tile_iter = 0;
+            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tile_iter) {
+                int tm, tn;
+                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+                const int sb = tile_iter & 1;
+                // the scales of this tile were copied by all epilogue threads during the
+                // previous tile
+                if (!mbar_wait(&sm.sready[sb], (tile_iter >> 1) & 1, abort))
+                    break;
+                const int tnext = t + gridDim.x;
+                if (tnext < p.num_tiles) {
+                    int tm2, tn2;
+                    tile_coords(tnext, p.num_tm, p.num_tn, tm2, tn2);
+                    scales_fetch(sm.sx[sb ^ 1], sm.sw[sb ^ 1], p, tm2, tn2, etid, kEpiThreads);
+                }
+                float2 acc[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    acc[j] = make_float2(0.0f, 0.0f);
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t buf = acc_i & 1;
+                    if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float sc = sm.sx[sb][kb] * sm.sw[sb][half][kb];   // FP32 scale product
+                    const float2 sc2 = make_float2(sc, sc);
+                    const float2 nmg = make_float2(-kAccInitF, -kAccInitF);
+                    const uint32_t tb = lane_base + buf * BN;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t r[16];
+                        tmem_ld16(tb + c * 16, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float2 v = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                            v = __fadd2_rn(v, nmg);                         // float(P), exact
+                            acc[c * 8 + j] = __ffma2_rn(v, sc2, acc[c * 8 + j]);
+                        }
+                        tmem_st16(tb + c * 16, fill);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&sm.tempty[buf]);
+                    ++acc_i;
+                }
+                if (!ok)
+                    break;
+                cp_async_wait_all();
+                mbar_arrive(&sm.sready[sb ^ 1]);
+                // bias + BF16 store: this thread owns row m, columns n0 .. n0 + 127
+                const int64_t m = static_cast<int64_t>(tm) * BM + row;
+                const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                if (n0 < p.N) {
+                    uint16_t *dst = p.y + m * p.N + n0;
+#pragma unroll
+                    for (int c8 = 0; c8 < 16; ++c8) {
+                        float bb[8];
+                        if (p.bias != nullptr) {
+                            const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + n0 + c8 * 8));
+                            bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
+                            bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
+                            bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
+                            bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                bb[i] = 0.0f;
+                        }
+                        uint4 o;
+                        o.x = pack_bf16x2(acc[c8 * 4 + 0].x + bb[0], acc[c8 * 4 + 0].y + bb[1]);
+                        o.y = pack_bf16x2(acc[c8 * 4 + 1].x + bb[2], acc[c8 * 4 + 1].y + bb[3]);
+                        o.z = pack_bf16x2(acc[c8 * 4 + 2].x + bb[4], acc[c8 * 4 + 2].y + bb[5]);
+                        o.w = pack_bf16x2(acc[c8 * 4 + 3].x + bb[6], acc[c8 * 4 + 3].y + bb[7]);
+                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = o;
+                    }
+                }
+            }
+        } else if (kMode == Mode::kI8Dump) {
+            const int KB = static_cast<int>(p.K / 128);
+            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+                const int64_t m = static_cast<int64_t>(tm) * BM + row;
+                const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t buf = acc_i & 1;
+                    if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tb = lane_base + buf * BN;
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tb + c * 32, r);
+                        tmem_wait_ld();
+                        if (n0 < p.N) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const float v = __uint_as_float(r[j]) - kAccInitF;
+                                p.dump[(m * p.N + n0 + c * 32 + j) * KB + kb] = static_cast<int32_t>(v);
+                            }
+                        }
+                        tmem_st16(tb + c * 32, fill);
+                        tmem_st16(tb + c * 32 + 16, fill);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&sm.tempty[buf]);
+                    ++acc_i;
+                }
+                if (!ok)
+                    break;
+            }
+        } else {
+            // BF16: one accumulator per tile, read once at the end of the tile.
+            const bool vec_ok = (p.N % 8) == 0;
+            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+                const uint32_t buf = acc_i & 1;
+                if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
+                    break;
+                tc_fence_after();
+                const int64_t m = static_cast<int64_t>(tm) * BM + row;
+                const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                const uint32_t tb = lane_base + buf * BN;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tb + c * 32, r);
+                    tmem_wait_ld();
+                    const int64_t nc = n0 + c * 32;
+                    if (m < p.M && nc < p.N) {
+                        uint16_t *dst = p.y + m * p.N + nc;
+                        if (vec_ok && nc + 32 <= p.N) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                float v[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    v[i] = __uint_as_float(r[g * 8 + i]);
+                                    if (p.bias != nullptr)
+                                        v[i] += __uint_as_float(static_cast<uint32_t>(p.bias[nc + g * 8 + i]) << 16);
+                                }
+                                uint4 o;
+                                o.x = pack_bf16x2(v[0], v[1]);
+                                o.y = pack_bf16x2(v[2], v[3]);
+                                o.z = pack_bf16x2(v[4], v[5]);
+                                o.w = pack_bf16x2(v[6], v[7]);
+                                *reinterpret_cast<uint4 *>(dst + g * 8) = o;
+                            }
+                        } else {
+                            for (int i = 0; i < 32 && nc + i < p.N; ++i) {
+                                float v = __uint_as_float(r[i]);
+                                if (p.bias != nullptr)
+                                    v += __uint_as_float(static_cast<uint32_t>(p.bias[nc + i]) << 16);
+                                dst[i] = static_cast<uint16_t>(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.tempty[buf]);
+                ++acc_i;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ CUDA-core fallback
+// y = x w^T + bias for any shape, alignment or K (including K = 0): 64 x 64 output tile
+// per 256-thread CTA, 4 x 4 outputs per thread, FP32 accumulation, K staged through
+// shared memory 16 at a time.  Used only when the tensor-core kernel cannot take the
+// buffers (K not a multiple of 8, or unaligned pointers).
+__global__ void __launch_bounds__(256) bf16_gemm_simt_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ w,
+    const uint16_t *__restrict__ bias, uint16_t *__restrict__ y, int64_t M, int64_t K, int64_t N)
+{
+    __shared__ float xs[16][64 + 1];
+    __shared__ float wsh[16][64 + 1];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * 64;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 64;
+    float acc[4][4] = {};
+    for (int64_t k0 = 0; k0 < K; k0 += 16) {
+        for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+            const int kk = i & 15, rr = i >> 4;
+            const int64_t gm = m0 + rr, gn = n0 + rr, gk = k0 + kk;
+            xs[kk][rr] = (gm < M && gk < K) ? __uint_as_float(static_cast<uint32_t>(x[gm * K + gk]) << 16) : 0.0f;
+            wsh[kk][rr] = (gn < N && gk < K) ? __uint_as_float(static_cast<uint32_t>(w[gn * K + gk]) << 16) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = xs[kk][ty * 4 + i];
+                b[i] = wsh[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t gm = m0 + ty * 4 + i;
+        if (gm >= M)
+            continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t gn = n0 + tx * 4 + j;
+            if (gn >= N)
+                continue;
+            float v = acc[i][j];
+            if (bias != nullptr)
+                v += __uint_as_float(static_cast<uint32_t>(bias[gn]) << 16);
+            y[gm * N + gn] = static_cast<uint16_t>(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+        }
+    }
+}
+
+} // namespace gemm
+} // namespace w8a8

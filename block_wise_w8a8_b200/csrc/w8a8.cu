@@ -1,0 +1,489 @@
+// w8a8.cu -- the C ABI of libw8a8 (declared in include/w8a8.h): argument checks, the
+// guard of the TurboT2VA paper's inference-stack section (guard paragraph: INT8 only for
+// CUDA BF16 inputs with flattened M, K, N divisible by 128, else a BF16 linear on the
+// retained BF16 weight), TMA descriptor set-up and kernel launches.  Everything is
+// enqueued on the caller's stream; nothing is allocated.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/w8a8.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace w8a8;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    bool gemm_attr_set[3] = {false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+w8a8_status_t current_device(int &dev)
+{
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev[dev].ready) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return W8A8_ERR_CUDA;
+        }
+        g_dev[dev].sms = sms;
+        g_dev[dev].ready = true;
+    }
+    return W8A8_OK;
+}
+
+w8a8_status_t get_encoder()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode != nullptr)
+        return W8A8_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return W8A8_OK;
+}
+
+// A buffer that kernels on the current device may read/write: device or managed memory
+// of this device.
+w8a8_status_t check_device_ptr(const void *p)
+{
+    if (p == nullptr)
+        return W8A8_ERR_INVALID_ARG;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_NOT_DEVICE;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+        return W8A8_ERR_NOT_DEVICE;
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (a.type == cudaMemoryTypeDevice && a.device != dev)
+        return W8A8_ERR_NOT_DEVICE;
+    return W8A8_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+w8a8_status_t cuda_fail(cudaError_t e)
+{
+    t_last_cuda_error = e;
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+}
+
+w8a8_status_t launch_status()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? W8A8_OK : cuda_fail(e);
+}
+
+#define W8A8_TRY(expr)                                                                   \
+    do {                                                                                 \
+        const w8a8_status_t st_ = (expr);                                                \
+        if (st_ != W8A8_OK)                                                              \
+            return st_;                                                                  \
+    } while (0)
+
+// Row-major [rows, cols] matrix of `es`-byte elements; box of box_rows x (128 bytes).
+w8a8_status_t make_map(CUtensorMap &m, const void *base, CUtensorMapDataType dt, int es,
+                       int64_t rows, int64_t cols, uint32_t box_rows)
+{
+    W8A8_TRY(get_encoder());
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * es};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(&m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+template <gemm::Mode kMode>
+w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
+                          cudaStream_t stream)
+{
+    int dev;
+    W8A8_TRY(current_device(dev));
+    constexpr bool kInt8 = kMode != gemm::Mode::kBf16;
+    CUtensorMap ta, tb;
+    const CUtensorMapDataType dt = kInt8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int es = kInt8 ? 1 : 2;
+    W8A8_TRY(make_map(ta, a, dt, es, p0.M, p0.K, gemm::BM));
+    W8A8_TRY(make_map(tb, b, dt, es, p0.N, p0.K, gemm::BN));
+    gemm::Params p = p0;
+    p.num_tm = static_cast<int32_t>((p.M + gemm::BM - 1) / gemm::BM);
+    p.num_tn = static_cast<int32_t>((p.N + gemm::BN - 1) / gemm::BN);
+    p.num_tiles = p.num_tm * p.num_tn;
+    const int64_t slice = kInt8 ? 128 : 64;
+    p.kslices = static_cast<int32_t>((p.K + slice - 1) / slice);
+    auto kern = gemm::gemm_kernel<kMode>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].gemm_attr_set[static_cast<int>(kMode)]) {
+            const cudaError_t e = cudaFuncSetAttribute(
+                kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(gemm::kSmemBytes));
+            if (e != cudaSuccess)
+                return cuda_fail(e);
+            // The kernel re-splits its registers between warpgroups (setmaxnreg); that
+            // split must fit in what the launch provides or the increase would never be
+            // granted.  Refuse to launch a build whose register count is too low.
+            cudaFuncAttributes fa;
+            const cudaError_t e2 = cudaFuncGetAttributes(&fa, kern);
+            if (e2 != cudaSuccess)
+                return cuda_fail(e2);
+            if (fa.numRegs * gemm::NUM_THREADS <
+                128 * gemm::kRegsControl + 256 * gemm::kRegsEpilogue)
+                return cuda_fail(cudaErrorInvalidConfiguration);
+            g_dev[dev].gemm_attr_set[static_cast<int>(kMode)] = true;
+        }
+    }
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, g_dev[dev].sms));
+    kern<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, stream>>>(ta, tb, p);
+    return launch_status();
+}
+
+w8a8_status_t quantize_impl(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
+                            cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0)
+        return W8A8_ERR_INVALID_ARG;
+    if (rows % 128 || cols % 128)
+        return W8A8_ERR_SHAPE;
+    if (rows == 0 || cols == 0)
+        return W8A8_OK;
+    W8A8_TRY(check_device_ptr(x));
+    W8A8_TRY(check_device_ptr(q));
+    W8A8_TRY(check_device_ptr(s));
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u))
+        return W8A8_ERR_ALIGNMENT;
+    int dev;
+    W8A8_TRY(current_device(dev));
+    const int64_t KB = cols / 128;
+    const int64_t nblocks = (rows / 128) * KB;
+    const int64_t grid = std::min<int64_t>(nblocks, static_cast<int64_t>(g_dev[dev].sms) * 8);
+    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kThreads, 0, stream>>>(
+        x, cols, nblocks, KB, q, s);
+    return launch_status();
+}
+
+size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+bool int8_shape_ok(int64_t M, int64_t K, int64_t N)
+{
+    return M > 0 && K > 0 && N > 0 && M % 128 == 0 && K % 128 == 0 && N % 128 == 0 &&
+           K <= 128 * gemm::KB_MAX;
+}
+
+w8a8_status_t check_weight(const w8a8_weight_t *w, int64_t K)
+{
+    if (w == nullptr || w->w_bf16 == nullptr || w->N < 0 || w->K != K)
+        return W8A8_ERR_INVALID_ARG;
+    if ((w->wq == nullptr) != (w->ws == nullptr))
+        return W8A8_ERR_INVALID_ARG;
+    return W8A8_OK;
+}
+
+w8a8_status_t gemm_i8_impl(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                           const w8a8_weight_t *w, const uint16_t *bias, uint16_t *y,
+                           cudaStream_t stream)
+{
+    gemm::Params p{};
+    p.M = M;
+    p.N = w->N;
+    p.K = K;
+    p.xs = xs;
+    p.ws = w->ws;
+    p.bias = bias;
+    p.y = y;
+    return launch_gemm<gemm::Mode::kI8Scaled>(xq, w->wq, p, stream);
+}
+
+w8a8_status_t bf16_impl(const uint16_t *x, const uint16_t *w, const uint16_t *bias, uint16_t *y,
+                        int64_t M, int64_t K, int64_t N, cudaStream_t stream)
+{
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    const bool tc = K > 0 && K % 8 == 0 && aligned16(x) && aligned16(w) && aligned16(y);
+    if (tc) {
+        gemm::Params p{};
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.bias = bias;
+        p.y = y;
+        return launch_gemm<gemm::Mode::kBf16>(x, w, p, stream);
+    }
+    const dim3 grid(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+    if (grid.y > 65535u)
+        return W8A8_ERR_SHAPE;
+    gemm::bf16_gemm_simt_kernel<<<grid, 256, 0, stream>>>(x, w, bias, y, M, K, N);
+    return launch_status();
+}
+
+__global__ void wait_timeout_kernel(uint64_t timeout_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        mbar_wait(&bar, 0, &abort_flag, timeout_ns);   // nothing ever arrives
+}
+
+} // namespace
+
+extern "C" {
+
+w8a8_status_t w8a8_quantize_weight(const w8a8_bf16_t *w, int64_t N, int64_t K, int8_t *wq,
+                                   float *ws, void *stream)
+{
+    if (N == 0 || K == 0)
+        return (N % 128 || K % 128 || N < 0 || K < 0) ? W8A8_ERR_SHAPE : W8A8_OK;
+    return quantize_impl(w, N, K, wq, ws, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_quantize_act(const w8a8_bf16_t *x, int64_t M, int64_t K, int8_t *xq,
+                                float *xs, void *stream)
+{
+    return quantize_impl(x, M, K, xq, xs, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
+                                        float eps, int64_t M, int64_t K, int8_t *xq, float *xs,
+                                        float *rstd_out, void *stream)
+{
+    if (M < 0 || K < 0 || !(eps >= 0.0f))
+        return W8A8_ERR_INVALID_ARG;
+    if (M % 128 || K % 128 || K > 16384)
+        return W8A8_ERR_SHAPE;
+    if (M == 0)
+        return W8A8_OK;
+    if (K == 0)
+        return W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(x));
+    W8A8_TRY(check_device_ptr(gamma));
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(xs));
+    if (rstd_out != nullptr)
+        W8A8_TRY(check_device_ptr(rstd_out));
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(xq) ||
+        (reinterpret_cast<uintptr_t>(xs) & 3u) || (reinterpret_cast<uintptr_t>(rstd_out) & 3u))
+        return W8A8_ERR_ALIGNMENT;
+    int dev;
+    W8A8_TRY(current_device(dev));
+    const int64_t MB = M / 128;
+    int max_clusters = 0;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(quant::kNormCluster * 64, 1, 1);
+        cfg.blockDim = dim3(quant::kThreads, 1, 1);
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = quant::kNormCluster;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, quant::rmsnorm_quantize_kernel, &cfg) !=
+                cudaSuccess ||
+            max_clusters <= 0) {
+            cudaGetLastError();
+            max_clusters = g_dev[dev].sms / quant::kNormCluster;
+        }
+    }
+    const int64_t nclusters = std::max<int64_t>(1, std::min<int64_t>(MB, max_clusters));
+    quant::rmsnorm_quantize_kernel<<<static_cast<unsigned>(nclusters * quant::kNormCluster),
+                                     quant::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        x, gamma, eps, MB, K, xq, xs, rstd_out);
+    return launch_status();
+}
+
+size_t w8a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N)
+{
+    if (!int8_shape_ok(M, K, N))
+        return 0;
+    return round256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+           static_cast<size_t>(M / 128) * static_cast<size_t>(K / 128) * sizeof(float);
+}
+
+w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8_weight_t *w,
+                          const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *workspace,
+                          size_t workspace_bytes, int *path_taken, void *stream)
+{
+    if (path_taken != nullptr)
+        *path_taken = W8A8_PATH_NONE;
+    if (M < 0 || K < 0)
+        return W8A8_ERR_INVALID_ARG;
+    W8A8_TRY(check_weight(w, K));
+    const int64_t N = w->N;
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K > 0)
+        W8A8_TRY(check_device_ptr(x));
+    W8A8_TRY(check_device_ptr(y));
+    if (K > 0)
+        W8A8_TRY(check_device_ptr(w->w_bf16));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    const bool int8 = int8_shape_ok(M, K, N) && w->wq != nullptr && aligned16(x) &&
+                      aligned16(y) && aligned16(w->wq) && aligned16(workspace) &&
+                      (bias == nullptr || aligned16(bias));
+    if (int8) {
+        W8A8_TRY(check_device_ptr(w->wq));
+        W8A8_TRY(check_device_ptr(w->ws));
+        const size_t need = w8a8_linear_workspace_bytes(M, K, N);
+        if (workspace == nullptr || workspace_bytes < need)
+            return W8A8_ERR_WORKSPACE;
+        W8A8_TRY(check_device_ptr(workspace));
+        int8_t *xq = static_cast<int8_t *>(workspace);
+        float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                              round256(static_cast<size_t>(M) * K));
+        W8A8_TRY(quantize_impl(x, M, K, xq, xs, st));
+        W8A8_TRY(gemm_i8_impl(xq, xs, M, K, w, bias, y, st));
+        if (path_taken != nullptr)
+            *path_taken = W8A8_PATH_INT8;
+        return W8A8_OK;
+    }
+    W8A8_TRY(bf16_impl(x, w->w_bf16, bias, y, M, K, N, st));
+    if (path_taken != nullptr)
+        *path_taken = W8A8_PATH_BF16;
+    return W8A8_OK;
+}
+
+w8a8_status_t w8a8_linear_prequant(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                                   const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                   w8a8_bf16_t *y, void *stream)
+{
+    if (M < 0 || K < 0)
+        return W8A8_ERR_INVALID_ARG;
+    W8A8_TRY(check_weight(w, K));
+    if (w->wq == nullptr)
+        return W8A8_ERR_INVALID_ARG;
+    if (M == 0 || w->N == 0)
+        return W8A8_OK;
+    if (!int8_shape_ok(M, K, w->N))
+        return W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(xs));
+    W8A8_TRY(check_device_ptr(w->wq));
+    W8A8_TRY(check_device_ptr(w->ws));
+    W8A8_TRY(check_device_ptr(y));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    if (!aligned16(xq) || !aligned16(w->wq) || !aligned16(y) || (bias && !aligned16(bias)))
+        return W8A8_ERR_ALIGNMENT;
+    return gemm_i8_impl(xq, xs, M, K, w, bias, y, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_bf16_linear(const w8a8_bf16_t *x, const w8a8_bf16_t *w,
+                               const w8a8_bf16_t *bias, w8a8_bf16_t *y, int64_t M, int64_t K,
+                               int64_t N, void *stream)
+{
+    if (M < 0 || K < 0 || N < 0)
+        return W8A8_ERR_INVALID_ARG;
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    if (K > 0) {
+        W8A8_TRY(check_device_ptr(x));
+        W8A8_TRY(check_device_ptr(w));
+    }
+    W8A8_TRY(check_device_ptr(y));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    return bf16_impl(x, w, bias, y, M, K, N, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_debug_block_sums(const int8_t *xq, const int8_t *wq, int64_t M, int64_t K,
+                                    int64_t N, int32_t *out, void *stream)
+{
+    if (M < 0 || K < 0 || N < 0)
+        return W8A8_ERR_INVALID_ARG;
+    if (!int8_shape_ok(M, K, N))
+        return W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(wq));
+    W8A8_TRY(check_device_ptr(out));
+    if (!aligned16(xq) || !aligned16(wq))
+        return W8A8_ERR_ALIGNMENT;
+    gemm::Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.dump = out;
+    return launch_gemm<gemm::Mode::kI8Dump>(xq, wq, p, static_cast<cudaStream_t>(stream));
+}
+
+int w8a8_device_error(void)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return v;
+}
+
+w8a8_status_t w8a8_debug_wait_timeout(uint64_t timeout_ns, void *stream)
+{
+    if (timeout_ns > 5000000000ull)
+        return W8A8_ERR_INVALID_ARG;
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return launch_status();
+}
+
+const char *w8a8_last_cuda_error(void)
+{
+    return cudaGetErrorString(t_last_cuda_error);
+}
+
+const char *w8a8_status_string(w8a8_status_t status)
+{
+    switch (status) {
+    case W8A8_OK: return "ok";
+    case W8A8_ERR_INVALID_ARG: return "invalid argument";
+    case W8A8_ERR_SHAPE: return "shape not supported by this entry point";
+    case W8A8_ERR_NOT_DEVICE: return "buffer is not device memory of the current device";
+    case W8A8_ERR_ALIGNMENT: return "buffer not 16-byte aligned";
+    case W8A8_ERR_WORKSPACE: return "workspace missing or too small";
+    case W8A8_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+} // extern "C"

@@ -1,0 +1,182 @@
+/*
+ * w8a8.h -- C ABI of the B200 (sm_100a) guarded block-wise W8A8 linear layer.
+ *
+ * The operation (TurboDiffusion article, bjdmk.com.cn news 725942, section
+ * "训练与推理的极致效率", inference list items 3-4; TurboT2VA paper, "TurboT2VA: Fast
+ * Large-Scale Text-to-Video-Audio Generation via Score-Regularized Consistency
+ * Distillation", inference-stack section, W8A8 operator and guard paragraphs):
+ *
+ *   X[M,K] (BF16) and W[N,K] (BF16, nn.Linear layout: row n is output channel n) are cut
+ *   into 128x128 blocks.  Each block gets one FP32 scale s = max|block| / 127 (s = 1 for an
+ *   all-zero block) and INT8 codes q = clamp(round_half_even(v / s), -127, 127), where
+ *   v / s is an IEEE FP32 division.  Weights are quantized once ("static"), activations on
+ *   every call.  The output is
+ *
+ *     Y[m,n] = bf16( sum_kb float(P[m,n,kb]) * (xs[m/128,kb] * ws[n/128,kb]) + bias[n] ),
+ *     P[m,n,kb] = sum_{k = 128 kb}^{128 kb + 127} xq[m,k] * wq[n,k]   (exact INT32),
+ *
+ *   i.e. the INT32 partial product of each 128-wide K block is rescaled by the two FP32
+ *   block scales before the blocks are summed in FP32.
+ *
+ *   Guard (TurboT2VA paper, guard paragraph): the INT8 path runs only for BF16 device
+ *   buffers whose flattened M, K and N are all multiples of 128; every other shape runs a
+ *   BF16 GEMM on the retained BF16 weight.  There is no CPU path.
+ *
+ * Conventions for every entry point:
+ *   - All matrices are row-major and contiguous.  BF16 values are passed as uint16_t
+ *     bit patterns (w8a8_bf16_t).  Sizes are element counts.
+ *   - Every buffer is owned by the caller and must be device memory (cudaMalloc /
+ *     PyTorch CUDA tensors) on the current device.  The library allocates no device
+ *     memory and keeps no state between calls other than a small host-side cache.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work is
+ *     enqueued on it and the call returns without waiting: outputs are ready once the
+ *     stream reaches that point.
+ *   - Argument errors are reported synchronously by the return code, before anything is
+ *     enqueued.  A failed launch returns W8A8_ERR_CUDA.  Faults inside a kernel surface
+ *     through the CUDA runtime as usual.  Every wait inside the kernels gives up after
+ *     about two seconds; the kernel then records W8A8_DEVERR_TIMEOUT in a device word
+ *     that w8a8_device_error() reads and clears.
+ *   - Outputs must not overlap inputs.
+ */
+#ifndef W8A8_H_
+#define W8A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W8A8_API __attribute__((visibility("default")))
+#else
+#define W8A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t w8a8_bf16_t;   /* bfloat16 bit pattern */
+
+typedef enum {
+    W8A8_OK = 0,
+    W8A8_ERR_INVALID_ARG = 1,   /* NULL pointer where one is required, negative size  */
+    W8A8_ERR_SHAPE = 2,         /* a 128-multiple was required and not given          */
+    W8A8_ERR_NOT_DEVICE = 3,    /* a buffer is host memory or on another device       */
+    W8A8_ERR_ALIGNMENT = 4,     /* a buffer is not 16-byte aligned                     */
+    W8A8_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required          */
+    W8A8_ERR_CUDA = 6           /* a CUDA runtime call or a launch failed              */
+} w8a8_status_t;
+
+typedef enum {
+    W8A8_PATH_INT8 = 0,         /* quantize activations + INT8 block-scaled GEMM       */
+    W8A8_PATH_BF16 = 1,         /* guard rejected the shape: BF16 GEMM                 */
+    W8A8_PATH_NONE = 2          /* nothing to compute (M == 0 or N == 0)               */
+} w8a8_path_t;
+
+/* Device-side error codes read by w8a8_device_error(). */
+#define W8A8_DEVERR_NONE 0
+#define W8A8_DEVERR_TIMEOUT 1   /* a bounded wait inside a kernel gave up              */
+
+/* A linear layer's weight as the caller keeps it.
+ *   w_bf16: [N, K] BF16, always required (the fallback GEMM uses it; the guard
+ *           paragraph's "retained BF16 weight copy").
+ *   wq:     [N, K] INT8 codes from w8a8_quantize_weight, or NULL when N or K is not a
+ *           multiple of 128 (the layer then always takes the BF16 path).
+ *   ws:     [N/128, K/128] FP32 block scales, NULL exactly when wq is NULL. */
+typedef struct {
+    int64_t N;
+    int64_t K;
+    const w8a8_bf16_t *w_bf16;
+    const int8_t *wq;
+    const float *ws;
+} w8a8_weight_t;
+
+/* Block-wise 128x128 quantization of a weight, done once when the layer is loaded.
+ *   w [N, K] BF16 -> wq [N, K] INT8 and ws [N/128, K/128] FP32 (row-major).
+ *   N and K must be positive multiples of 128 (else W8A8_ERR_SHAPE); all three buffers
+ *   16-byte aligned.  Same arithmetic as w8a8_quantize_act. */
+W8A8_API w8a8_status_t w8a8_quantize_weight(const w8a8_bf16_t *w, int64_t N, int64_t K, int8_t *wq,
+                                   float *ws, void *stream);
+
+/* Block-wise 128x128 dynamic quantization of activations (TurboDiffusion article,
+ * inference list item 4: activations quantized at the weights' block granularity).
+ *   x [M, K] BF16 -> xq [M, K] INT8 and xs [M/128, K/128] FP32.
+ *   M and K multiples of 128 (else W8A8_ERR_SHAPE; M == 0 is a no-op); 16-byte aligned.
+ *   Reads x once and writes xq, xs once. */
+W8A8_API w8a8_status_t w8a8_quantize_act(const w8a8_bf16_t *x, int64_t M, int64_t K, int8_t *xq,
+                                float *xs, void *stream);
+
+/* RMSNorm fused ahead of the activation quantizer (TurboDiffusion article, inference
+ * list item 5: norm kernels re-implemented in CUDA; TurboT2VA paper, fused-operator
+ * paragraph).  For each row m:
+ *     rstd[m] = fp32( 1 / sqrt( (sum_k x[m,k]^2) / K + eps ) )   (sum and sqrt in FP64)
+ *     y[m,k]  = bf16( (x[m,k] * rstd[m]) * gamma[k] )            (FP32 products)
+ *   and y is block-quantized exactly as by w8a8_quantize_act, without being stored.
+ *   x [M, K] BF16, gamma [K] BF16 -> xq [M, K] INT8, xs [M/128, K/128] FP32, and
+ *   rstd_out [M] FP32 when not NULL.  M, K multiples of 128; K <= 16384. */
+W8A8_API w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
+                                        float eps, int64_t M, int64_t K, int8_t *xq,
+                                        float *xs, float *rstd_out, void *stream);
+
+/* Bytes of device workspace w8a8_linear needs for an M x K activation on the INT8 path:
+ * the INT8 codes (M*K bytes, rounded up to 256) followed by the FP32 scales.  Returns 0
+ * when the shape takes the BF16 path. */
+W8A8_API size_t w8a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
+
+/* The guarded W8A8 linear: Y[M, N] = X[M, K] W^T + bias, BF16 out.
+ *   x:    [M, K] BF16 device buffer (flattened leading dimensions).
+ *   w:    host pointer to the weight record (the buffers it names are device memory).
+ *   bias: [N] BF16 or NULL.
+ *   y:    [M, N] BF16.
+ *   workspace: device buffer of at least w8a8_linear_workspace_bytes(M, K, N) bytes,
+ *          used for the quantized activations; may be NULL when that size is 0.
+ *   path_taken: if not NULL, receives the w8a8_path_t that ran.
+ * Guard: INT8 path iff M, K, N > 0 and all multiples of 128, K <= 65536, w->wq and
+ * w->ws are present, and x, y, wq, workspace are 16-byte aligned.  Otherwise the BF16
+ * GEMM runs on w->w_bf16 (any M, K, N >= 0; K == 0 gives y = bias or 0). */
+W8A8_API w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8_weight_t *w,
+                          const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *workspace,
+                          size_t workspace_bytes, int *path_taken, void *stream);
+
+/* The INT8 GEMM with per-K-block rescale on activations that are already quantized
+ * (e.g. by w8a8_rmsnorm_quantize_act).  xq [M, K] INT8, xs [M/128, K/128] FP32, the
+ * weight's wq/ws, bias [N] or NULL, y [M, N] BF16.  M, K, N multiples of 128
+ * (else W8A8_ERR_SHAPE); K <= 65536. */
+W8A8_API w8a8_status_t w8a8_linear_prequant(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                                   const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                   w8a8_bf16_t *y, void *stream);
+
+/* The BF16 GEMM that the guard falls back to, callable directly:
+ *   y[M, N] = bf16( sum_k x[m,k] w[n,k] (FP32 accumulation) + bias[n] ).
+ *   Any M, K, N >= 0.  Uses tcgen05 tensor cores when K is a multiple of 8 and the
+ *   buffers are 16-byte aligned, else a CUDA-core kernel. */
+W8A8_API w8a8_status_t w8a8_bf16_linear(const w8a8_bf16_t *x, const w8a8_bf16_t *w,
+                               const w8a8_bf16_t *bias, w8a8_bf16_t *y, int64_t M, int64_t K,
+                               int64_t N, void *stream);
+
+/* Test hook: the INT32 partial products P[m, n, kb] of the INT8 GEMM, written by the
+ * same tensor-core main loop as w8a8_linear, for xq [M, K] and wq [N, K] (M, K, N
+ * multiples of 128).  out: [M, N, K/128] INT32 device buffer. */
+W8A8_API w8a8_status_t w8a8_debug_block_sums(const int8_t *xq, const int8_t *wq, int64_t M, int64_t K,
+                                    int64_t N, int32_t *out, void *stream);
+
+/* Synchronizes the current device and returns (and clears) the device error word:
+ * W8A8_DEVERR_NONE or W8A8_DEVERR_TIMEOUT. */
+W8A8_API int w8a8_device_error(void);
+
+/* Test hook for the bounded waits: launches one CTA that waits on a barrier nothing
+ * arrives on, giving up after timeout_ns nanoseconds; the device error word then reads
+ * W8A8_DEVERR_TIMEOUT.  Touches no caller memory. */
+W8A8_API w8a8_status_t w8a8_debug_wait_timeout(uint64_t timeout_ns, void *stream);
+
+/* The CUDA runtime's description of the last CUDA error that made a call of this thread
+ * return W8A8_ERR_CUDA ("no error" if none).  Static storage; do not free. */
+W8A8_API const char *w8a8_last_cuda_error(void);
+
+/* A short static description of a status code. */
+W8A8_API const char *w8a8_status_string(w8a8_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H_ */

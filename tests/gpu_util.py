@@ -1,0 +1,31 @@
+"""Helpers shared by the GPU tests: moving BF16 bit patterns between numpy and torch,
+and the output tolerance of the W8A8 linear."""
+import numpy as np
+import torch
+
+RTOL = 1e-2
+ATOL = 1e-2
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_bits(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_to_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def assert_close_bf16(y_gpu_bits, ref_f32, orc, what=""):
+    """|y - bf16(ref)| <= ATOL + RTOL * |bf16(ref)| elementwise (ref = oracle FP32 output)."""
+    ref_b = bf16_to_f32(orc.f32_to_bf16(ref_f32)).astype(np.float64)
+    y = bf16_to_f32(y_gpu_bits).astype(np.float64)
+    err = np.abs(y - ref_b)
+    lim = ATOL + RTOL * np.abs(ref_b)
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
+                           f"worst err {float(err.max())} at {np.unravel_index(np.argmax(err - lim), err.shape)}")
+    return float(err.max()), float((err / (np.abs(ref_b) + 1e-30)).max())

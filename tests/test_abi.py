@@ -1,0 +1,68 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the header
+declares, the header compiles as plain C, and the size query needs no device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w8a8.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w8a8_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import block_wise_w8a8_b200.build as b
+    b.build()
+    return ctypes.CDLL(b.LIB)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 11, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in w8a8.h but not exported"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import block_wise_w8a8_b200.build as b
+    out = subprocess.run(["nm", "-D", "--defined-only", b.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted({line.split()[-1] for line in out.splitlines()
+                       if line.split()[-1].startswith("w8a8_")})
+    assert exported == _declared()
+
+
+def test_header_is_plain_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "w8a8.h"\nint main(void){ w8a8_weight_t w = {0}; (void)w; '
+                   'return (int)w8a8_linear_workspace_bytes(128, 128, 128) == 0; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only",
+                    "-I", os.path.join(ROOT, "include"), str(src)], check=True)
+
+
+def test_workspace_query_and_status_strings(lib):
+    lib.w8a8_linear_workspace_bytes.restype = ctypes.c_size_t
+    lib.w8a8_linear_workspace_bytes.argtypes = [ctypes.c_int64] * 3
+    assert lib.w8a8_linear_workspace_bytes(256, 384, 128) == 256 * 384 + 2 * 3 * 4
+    assert lib.w8a8_linear_workspace_bytes(1000, 2048, 8192) == 0      # guard: BF16 path
+    assert lib.w8a8_linear_workspace_bytes(1024, 2000, 8192) == 0
+    assert lib.w8a8_linear_workspace_bytes(128, 128, 100) == 0
+    lib.w8a8_status_string.restype = ctypes.c_char_p
+    assert lib.w8a8_status_string(0) == b"ok"
+    assert lib.w8a8_status_string(5).startswith(b"workspace")
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import block_wise_w8a8_b200 as w8
+    monkeypatch.setattr(w8, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(w8, "_lib", None)
+    with pytest.raises(RuntimeError):
+        w8.lib()
