@@ -44,6 +44,9 @@ _SIGS = {
     "w8a8_linear": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                     ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
+    "w8a8_linear_noalloc": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                            ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p,
+                            ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
     "w8a8_linear_prequant": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                              ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p,
                              ctypes.c_void_p],
@@ -186,6 +189,27 @@ def linear(x, weight, bias=None, out=None, workspace=None, return_path=False):
     _check("w8a8_linear", lib().w8a8_linear(
         _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
         0 if workspace is None else workspace.numel(), ctypes.byref(path), _stream(dev)))
+    return (out, path.value) if return_path else out
+
+
+NOALLOC_MAX_ELEMS = 16777216
+
+
+def linear_noalloc(x, weight, bias=None, out=None, return_path=False):
+    """w8a8_linear for callers that must not allocate device memory: the quantized
+    activations live in scratch built into the library (M * K <= 16 Mi on the INT8 path).
+    All calls on a device share that scratch, so calls that may overlap on the GPU must be
+    ordered (e.g. issued on one stream)."""
+    _need(x, torch.bfloat16, "x")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias")
+    K = x.shape[-1]
+    M = math.prod(x.shape[:-1])
+    dev = x.device
+    out = torch.empty((*x.shape[:-1], weight.N), dtype=torch.bfloat16, device=dev) if out is None else out
+    path = ctypes.c_int(-1)
+    _check("w8a8_linear_noalloc", lib().w8a8_linear_noalloc(
+        _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), ctypes.byref(path), _stream(dev)))
     return (out, path.value) if return_path else out
 
 

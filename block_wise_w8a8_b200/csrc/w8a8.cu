@@ -259,6 +259,36 @@ __global__ void wait_timeout_kernel(uint64_t timeout_ns)
         mbar_wait(&bar, 0, &abort_flag, timeout_ns);   // nothing ever arrives
 }
 
+// ------------------------------------------------------------------ no-allocation variant
+// Scratch for w8a8_linear_noalloc: the INT8 codes of the activations (first
+// W8A8_NOALLOC_MAX_ELEMS bytes) followed by their FP32 block scales.  It is a module
+// global, so every GPU that loads this library holds it until the process exits, and all
+// calls of w8a8_linear_noalloc on a device share it.
+constexpr size_t kNoAllocCodeBytes = static_cast<size_t>(W8A8_NOALLOC_MAX_ELEMS);
+constexpr size_t kNoAllocScaleBytes = (static_cast<size_t>(W8A8_NOALLOC_MAX_ELEMS) / (128 * 128)) * sizeof(float);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocCodeBytes + kNoAllocScaleBytes];
+
+// Host code cannot use g_noalloc_scratch's name as a device address; its address on each
+// device is looked up once, with that device current, and cached here.
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+w8a8_status_t noalloc_scratch(int dev, void *&ptr)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            t_last_cuda_error = e;
+            cudaGetLastError();
+            return W8A8_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    ptr = g_noalloc_ptr[dev];
+    return W8A8_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -377,6 +407,53 @@ w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8
     W8A8_TRY(bf16_impl(x, w->w_bf16, bias, y, M, K, N, st));
     if (path_taken != nullptr)
         *path_taken = W8A8_PATH_BF16;
+    return W8A8_OK;
+}
+
+w8a8_status_t w8a8_linear_noalloc(const w8a8_bf16_t *x, int64_t M, int64_t K,
+                                  const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                  w8a8_bf16_t *y, int *path_taken, void *stream)
+{
+    if (path_taken != nullptr)
+        *path_taken = W8A8_PATH_NONE;
+    if (M < 0 || K < 0)
+        return W8A8_ERR_INVALID_ARG;
+    W8A8_TRY(check_weight(w, K));
+    const int64_t N = w->N;
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    const bool int8 = int8_shape_ok(M, K, N) && w->wq != nullptr && aligned16(x) &&
+                      aligned16(y) && aligned16(w->wq) && (bias == nullptr || aligned16(bias));
+    if (!int8) {
+        // The BF16 fallback needs no scratch: same launch as w8a8_linear's fallback.
+        return w8a8_linear(x, M, K, w, bias, y, nullptr, 0, path_taken, stream);
+    }
+    if (M * K > static_cast<int64_t>(W8A8_NOALLOC_MAX_ELEMS))
+        return W8A8_ERR_WORKSPACE;
+    W8A8_TRY(check_device_ptr(x));
+    W8A8_TRY(check_device_ptr(y));
+    W8A8_TRY(check_device_ptr(w->wq));
+    W8A8_TRY(check_device_ptr(w->ws));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    int dev;
+    W8A8_TRY(current_device(dev));
+    void *scratch = nullptr;
+    W8A8_TRY(noalloc_scratch(dev, scratch));
+    // The quantize kernel rewrites every code and scale the GEMM then reads, so nothing in
+    // the scratch has to be cleared between calls.
+    int8_t *xq = static_cast<int8_t *>(scratch);
+    float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + kNoAllocCodeBytes);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t KB = K / 128;
+    const int64_t nblocks = (M / 128) * KB;
+    const int64_t grid = std::min<int64_t>(nblocks, static_cast<int64_t>(g_dev[dev].sms) * 8);
+    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kThreads, 0, st>>>(
+        x, K, nblocks, KB, xq, xs);
+    W8A8_TRY(launch_status());
+    W8A8_TRY(gemm_i8_impl(xq, xs, M, K, w, bias, y, st));
+    if (path_taken != nullptr)
+        *path_taken = W8A8_PATH_INT8;
     return W8A8_OK;
 }
 

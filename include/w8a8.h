@@ -137,6 +137,38 @@ W8A8_API w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, c
                           const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *workspace,
                           size_t workspace_bytes, int *path_taken, void *stream);
 
+/* Largest M * K that w8a8_linear_noalloc accepts on the INT8 path (16 Mi elements,
+ * e.g. M = K = 4096). */
+#define W8A8_NOALLOC_MAX_ELEMS (16777216LL)
+
+/* w8a8_linear for callers that cannot allocate device memory.  The paper has no
+ * counterpart to this entry point; it exists for users of this library.
+ *
+ * Some callers may not call cudaMalloc at all: code embedded in a host program that owns
+ * every byte of device memory through its own pool and forbids side allocations, or a
+ * latency-critical loop that cannot risk an allocation synchronizing the device or
+ * failing under memory pressure.  Such callers cannot provide w8a8_linear's workspace.
+ * This entry point computes exactly what w8a8_linear computes, with the same kernels and
+ * the same guard, but keeps the quantized activations in a fixed scratch array that is
+ * part of the library itself (16 MiB + 4 KiB of device memory, reserved on every GPU
+ * that loads the library and held until the process exits).  It calls no allocation
+ * routine.  The caller still passes x, the weight record, bias and y.
+ *
+ *   - INT8-path shapes with M * K > W8A8_NOALLOC_MAX_ELEMS are rejected with
+ *     W8A8_ERR_WORKSPACE before anything is enqueued.  Shapes that the guard sends to the
+ *     BF16 GEMM need no scratch and are not limited.
+ *   - The first call on each device looks up the scratch array's device address (with
+ *     that device current) and caches it; make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the one scratch array, and it keeps whatever the last
+ *     call wrote.  Nothing in it needs clearing (each call rewrites all it reads), but
+ *     calls whose work overlaps on the GPU (different streams, or different host threads,
+ *     without ordering between them) race on it and may produce wrong results: order such
+ *     calls, e.g. by issuing them on one stream. */
+W8A8_API w8a8_status_t w8a8_linear_noalloc(const w8a8_bf16_t *x, int64_t M, int64_t K,
+                                           const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                           w8a8_bf16_t *y, int *path_taken, void *stream);
+
 /* The INT8 GEMM with per-K-block rescale on activations that are already quantized
  * (e.g. by w8a8_rmsnorm_quantize_act).  xq [M, K] INT8, xs [M/128, K/128] FP32, the
  * weight's wq/ws, bias [N] or NULL, y [M, N] BF16.  M, K, N multiples of 128
