@@ -68,6 +68,36 @@ __device__ __forceinline__ uint2 quantize8(const uint32_t (&w)[4], float sc, flo
     return out;
 }
 
+// Fast codes of 8 BF16 values (as quantize8, without the exact fallback).  Bit i of the
+// returned `band` is set when value i's y lies within 2^-14 of a half-integer: its code
+// must then be taken from the IEEE division (code_exact) instead.
+__device__ __forceinline__ uint2 quantize8_fast(const uint32_t (&w)[4], float rc, uint32_t &band)
+{
+    uint32_t t[8];
+    uint32_t b = 0;
+    const float2 r2 = make_float2(rc, rc);
+    const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+    const float2 nmg = make_float2(-kRoundMagic, -kRoundMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 v = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
+        const float2 y = __fmul2_rn(v, r2);          // ~ v / s
+        const float2 tt = __fadd2_rn(y, mg);         // 1.5*2^23 + rne(y): low byte = code
+        const float2 n = __fadd2_rn(tt, nmg);        // rne(y), exact
+        const float2 d = __ffma2_rn(n, neg1, y);     // y - rne(y), exact, in [-0.5, 0.5]
+        b |= (fabsf(d.x) >= kTieBand ? 1u : 0u) << (2 * i);
+        b |= (fabsf(d.y) >= kTieBand ? 1u : 0u) << (2 * i + 1);
+        t[2 * i] = __float_as_uint(tt.x);
+        t[2 * i + 1] = __float_as_uint(tt.y);
+    }
+    band = b;
+    uint2 out;
+    out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    return out;
+}
+
 // Largest |BF16| among 8 values, as a BF16 magnitude pattern in the low 16 bits
 // (for finite values the magnitude order equals the unsigned order of the patterns).
 __device__ __forceinline__ uint32_t absmax8_bits(const uint32_t (&w)[4], uint32_t m)
@@ -98,40 +128,190 @@ __device__ __forceinline__ float block_scale_from(uint32_t m2, uint32_t *red)
     return (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
 }
 
-// x [rows, K] BF16 -> q [rows, K] INT8, s [rows/128, K/128] FP32.  Grid-stride over the
-// (rows/128) * (K/128) blocks.  Thread t covers rows (t / 16) + 16 i, i = 0..7, and the
-// 8 columns 8 (t % 16) .. + 7 of the block: a warp's 16-byte loads cover two full
-// 256-byte rows, its 8-byte stores two full 128-byte rows.
-__global__ void __launch_bounds__(kThreads) quantize_blocks_kernel(
-    const uint16_t *__restrict__ x, int64_t K, int64_t nblocks, int64_t KB,
-    int8_t *__restrict__ q, float *__restrict__ s)
+// ------------------------------------------------------------------ block quantizer ----
+// x [rows, K] BF16 -> q [rows, K] INT8, s [rows/128, K/128] FP32.
+//
+// Persistent: one CTA per SM takes the 128x128 blocks blockIdx.x + i gridDim.x,
+// i = 0, 1, ..., in row-major block order.  Warp 16 (one thread) streams them into a ring
+// of kQStages 32 KB shared-memory slots with 2-D TMA loads (no swizzle, no multicast),
+// which keeps up to kQStages blocks per SM in flight.  The 16 consumer warps form
+// kQGroups independent groups of 4; group g quantizes the CTA's blocks i = g, g + 4, ...,
+// so the latency chain of one block (absmax reduction, IEEE scale division, reciprocal)
+// overlaps the arithmetic of the other groups' blocks.  Within a group, thread t
+// (0..127) holds the 16-byte chunks t + 128 j, j = 0..15 (rows t / 16 + 8 j, columns
+// 8 (t % 16) .. + 7).  It reads them once to reduce the block's absmax (packed 16-bit
+// magnitudes, warp shuffles, then the 4 warp maxima through shared memory) and once more
+// to form the codes, which it writes with 8-byte stores (a warp covers two full 128-byte
+// rows of codes).  Every
+// wait is a bounded mbarrier wait; no named barrier is used.
+constexpr int kQStages = 6;
+constexpr int kQGroups = 4;                          // independent consumer groups
+constexpr int kQGroupWarps = 4;                      // warps per group
+constexpr int kQWarps = kQGroups * kQGroupWarps;    // consumer warps
+constexpr int kQChunks = 2048 / (kQGroupWarps * 32); // 16-byte chunks per thread per block
+constexpr int kQThreads = (kQWarps + 1) * 32;       // + the TMA producer warp
+constexpr uint32_t kQBlockBytes = 128 * 128 * 2;
+
+struct alignas(1024) QSmem {
+    uint16_t tile[kQStages][128 * 128];
+    uint64_t full[kQStages];
+    uint64_t empty[kQStages];
+    uint64_t red_full[kQGroups][2];
+    alignas(16) uint32_t red[kQGroups][2][kQGroupWarps];
+    int abort;
+};
+constexpr size_t kQSmemBytes = sizeof(QSmem) + 1024;
+static_assert(kQGroupWarps == 4, "the group's partial maxima are read as one 16-byte vector");
+static_assert(kQStages >= kQGroups, "every group needs a slot of its own");
+static_assert((2 * kQStages) % kQGroups == 0,
+              "item it - 2 S of the ring must belong to the same group as item it");
+
+__device__ __forceinline__ uint4 ld_shared_v4(const void *p)
 {
-    __shared__ uint32_t red[kThreads / 32];
-    const int rg = threadIdx.x >> 4;
-    const int cc = threadIdx.x & 15;
-    for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
-        const int64_t mb = blk / KB, kb = blk - mb * KB;
-        const int64_t off = (mb * 128 + rg) * K + kb * 128 + cc * 8;
-        uint32_t w[8][4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint4 v = ld_nc_v4(x + off + static_cast<int64_t>(i) * 16 * K);
-            w[i][0] = v.x; w[i][1] = v.y; w[i][2] = v.z; w[i][3] = v.w;
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__global__ void __launch_bounds__(kQThreads, 1)
+    quantize_blocks_kernel(const __grid_constant__ CUtensorMap tmX, int64_t K, int64_t nblocks,
+                           int64_t KB, int8_t *__restrict__ q, float *__restrict__ s)
+{
+    extern __shared__ uint8_t smem_raw[];
+    QSmem &sm = *reinterpret_cast<QSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kQGroupWarps);
         }
-        uint32_t m = 0;
+        for (int g = 0; g < kQGroups; ++g) {
+            mbar_init(&sm.red_full[g][0], kQGroupWarps);
+            mbar_init(&sm.red_full[g][1], kQGroupWarps);
+        }
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kQWarps) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmX);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
+                const uint32_t st = it % kQStages, ph = (it / kQStages) & 1;
+                if (!mbar_wait(&sm.empty[st], ph ^ 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                const int64_t mb = blk / KB, kb = blk - mb * KB;
+                mbar_arrive_expect_tx(&sm.full[st], kQBlockBytes);
+                tma_load_2d(sm.tile[st], &tmX, &sm.full[st], static_cast<int32_t>(kb * 128),
+                            static_cast<int32_t>(mb * 128));
+            }
+            if (!ok) {
+                // the copies already in flight land before shared memory is released
+                volatile int no_abort = 0;
+                const uint32_t first = it > kQStages ? it - kQStages : 0;
+                for (uint32_t j = first; j < it; ++j)
+                    mbar_wait(&sm.full[j % kQStages], (j / kQStages) & 1, &no_abort, 100000000ull);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int g = warp / kQGroupWarps;
+    const int gw = warp % kQGroupWarps;
+    const int gt = threadIdx.x % (kQGroupWarps * 32);
+    const int row0 = gt >> 4;
+    const int col = (gt & 15) * 8;
+    constexpr int kRowStep = kQGroupWarps * 32 / 16;     // rows between a thread's chunks
+    uint32_t gi = 0;                                     // this group's block count
+    for (int64_t blk = blockIdx.x + static_cast<int64_t>(g) * gridDim.x; blk < nblocks;
+         blk += static_cast<int64_t>(kQGroups) * gridDim.x, ++gi) {
+        const uint32_t it = gi * kQGroups + g;           // position in the ring's sequence
+        const uint32_t st = it % kQStages, ph = (it / kQStages) & 1;
+        // Slot st carries items it - S, it, it + S, ... of different groups.  A parity
+        // wait cannot tell phase p from p + 2, so first make sure item it - S has been
+        // consumed (the slot's full barrier is then in item it's phase or just past it).
+        // That wait is itself unambiguous: item it - 2S belongs to this group and is done.
+        if (it >= static_cast<uint32_t>(kQStages) && !mbar_wait(&sm.empty[st], ph ^ 1, abort))
+            break;
+        if (!mbar_wait(&sm.full[st], ph, abort))
+            break;
+        const uint16_t *tile = sm.tile[st];
+        // pass 1 over the tile: absmax (the tile is read again for the codes, which keeps
+        // the registers free while the group waits for the block's scale)
+        uint32_t m2 = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            m = absmax8_bits(w[i], m);
-        const float sc = block_scale_from(m, red);
+        for (int j = 0; j < kQChunks; ++j) {
+            const uint4 v = ld_shared_v4(tile + (row0 + kRowStep * j) * 128 + col);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            m2 = absmax8_bits(w, m2);
+        }
+        uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        const uint32_t rb = gi & 1;
+        if (lane == 0) {
+            sm.red[g][rb][gw] = m;
+            mbar_arrive(&sm.red_full[g][rb]);
+        }
+        if (!mbar_wait(&sm.red_full[g][rb], (gi >> 1) & 1, abort))
+            break;
+        const uint4 r4 = ld_shared_v4(&sm.red[g][rb][0]);
+        const uint32_t a = max(max(r4.x, r4.y), max(r4.z, r4.w));
+        const float amax = __uint_as_float(a << 16);
+        const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 127.0f);
         const float rc = __frcp_rn(sc);
-        const bool exact = !(rc <= 3.0e38f);
-        if (threadIdx.x == 0)
+        if (gt == 0)
             s[blk] = sc;
+        const int64_t mb = blk / KB, kb = blk - mb * KB;
+        int8_t *qb = q + (mb * 128 + row0) * K + kb * 128 + col;
+        uint32_t band[kQChunks / 4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<uint2 *>(q + off + static_cast<int64_t>(i) * 16 * K) =
-                quantize8(w[i], sc, rc, exact);
-        __syncthreads();
+        for (int j = 0; j < kQChunks; ++j) {
+            const uint4 v = ld_shared_v4(tile + (row0 + kRowStep * j) * 128 + col);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t bj;
+            *reinterpret_cast<uint2 *>(qb + static_cast<int64_t>(j) * kRowStep * K) =
+                quantize8_fast(w, rc, bj);
+            if ((j & 3) == 0)
+                band[j >> 2] = bj;
+            else
+                band[j >> 2] |= bj << (8 * (j & 3));
+        }
+        // Values near a half-integer (about 0.3% of N(0,1) BF16 data), and every value of
+        // a block whose 1/s overflows (s below about 2^-128), get their code from the
+        // division.  They are re-read from the tile and patched one byte at a time after
+        // the 8-byte stores above (same thread, same address: the later store wins).
+        const bool all_exact = !(rc <= 3.0e38f);
+#pragma unroll
+        for (int k = 0; k < kQChunks / 4; ++k) {
+            uint32_t b = all_exact ? 0xFFFFFFFFu : band[k];
+            while (b != 0) {
+                const int e = __ffs(b) - 1;
+                b &= b - 1;
+                const int j = 4 * k + (e >> 3);
+                const int r = row0 + kRowStep * j, c = col + (e & 7);
+                const float v = __uint_as_float(static_cast<uint32_t>(tile[r * 128 + c]) << 16);
+                qb[static_cast<int64_t>(j) * kRowStep * K + (e & 7)] =
+                    static_cast<int8_t>(code_exact(v, sc));
+            }
+        }
+        // every lane is done with the slot (its loads were consumed above)
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.empty[st]);
     }
 }
 

@@ -17,11 +17,14 @@ namespace {
 using namespace w8a8;
 
 constexpr int kMaxDevices = 64;
+// TMA coordinates are signed 32-bit: matrix extents stay below 2^31.
+constexpr int64_t kMaxTmaCoord = (int64_t{1} << 31) - 128;
 
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     bool gemm_attr_set[3] = {false, false, false};
+    bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -107,20 +110,30 @@ w8a8_status_t launch_status()
             return st_;                                                                  \
     } while (0)
 
-// Row-major [rows, cols] matrix of `es`-byte elements; box of box_rows x (128 bytes).
+// Row-major [rows, cols] matrix of `es`-byte elements; box of box_rows x box_cols
+// elements.
 w8a8_status_t make_map(CUtensorMap &m, const void *base, CUtensorMapDataType dt, int es,
-                       int64_t rows, int64_t cols, uint32_t box_rows)
+                       int64_t rows, int64_t cols, uint32_t box_rows, uint32_t box_cols,
+                       CUtensorMapSwizzle swizzle)
 {
     W8A8_TRY(get_encoder());
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * es};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode(&m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// GEMM operand: box of box_rows x 128 bytes, 128-byte swizzle (the UMMA K-major layout).
+w8a8_status_t make_operand_map(CUtensorMap &m, const void *base, CUtensorMapDataType dt,
+                               int es, int64_t rows, int64_t cols, uint32_t box_rows)
+{
+    return make_map(m, base, dt, es, rows, cols, box_rows, static_cast<uint32_t>(128 / es),
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <gemm::Mode kMode>
@@ -133,8 +146,8 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
     CUtensorMap ta, tb;
     const CUtensorMapDataType dt = kInt8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int es = kInt8 ? 1 : 2;
-    W8A8_TRY(make_map(ta, a, dt, es, p0.M, p0.K, gemm::BM));
-    W8A8_TRY(make_map(tb, b, dt, es, p0.N, p0.K, gemm::BN));
+    W8A8_TRY(make_operand_map(ta, a, dt, es, p0.M, p0.K, gemm::BM));
+    W8A8_TRY(make_operand_map(tb, b, dt, es, p0.N, p0.K, gemm::BN));
     gemm::Params p = p0;
     p.num_tm = static_cast<int32_t>((p.M + gemm::BM - 1) / gemm::BM);
     p.num_tn = static_cast<int32_t>((p.N + gemm::BN - 1) / gemm::BN);
@@ -167,12 +180,41 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
     return launch_status();
 }
 
+// Block quantization of x [rows, cols] (both multiples of 128, buffers already checked):
+// one persistent CTA per SM, blocks streamed in by TMA.
+w8a8_status_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
+                              cudaStream_t stream)
+{
+    int dev;
+    W8A8_TRY(current_device(dev));
+    CUtensorMap tm;
+    W8A8_TRY(make_map(tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].quant_attr_set) {
+            const cudaError_t e = cudaFuncSetAttribute(quant::quantize_blocks_kernel,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       static_cast<int>(quant::kQSmemBytes));
+            if (e != cudaSuccess)
+                return cuda_fail(e);
+            g_dev[dev].quant_attr_set = true;
+        }
+    }
+    const int64_t KB = cols / 128;
+    const int64_t nblocks = (rows / 128) * KB;
+    const int64_t grid = std::min<int64_t>(nblocks, g_dev[dev].sms);
+    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kQThreads,
+                                    quant::kQSmemBytes, stream>>>(tm, cols, nblocks, KB, q, s);
+    return launch_status();
+}
+
 w8a8_status_t quantize_impl(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
                             cudaStream_t stream)
 {
     if (rows < 0 || cols < 0)
         return W8A8_ERR_INVALID_ARG;
-    if (rows % 128 || cols % 128)
+    if (rows % 128 || cols % 128 || rows > kMaxTmaCoord || cols > kMaxTmaCoord)
         return W8A8_ERR_SHAPE;
     if (rows == 0 || cols == 0)
         return W8A8_OK;
@@ -181,14 +223,7 @@ w8a8_status_t quantize_impl(const uint16_t *x, int64_t rows, int64_t cols, int8_
     W8A8_TRY(check_device_ptr(s));
     if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u))
         return W8A8_ERR_ALIGNMENT;
-    int dev;
-    W8A8_TRY(current_device(dev));
-    const int64_t KB = cols / 128;
-    const int64_t nblocks = (rows / 128) * KB;
-    const int64_t grid = std::min<int64_t>(nblocks, static_cast<int64_t>(g_dev[dev].sms) * 8);
-    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kThreads, 0, stream>>>(
-        x, cols, nblocks, KB, q, s);
-    return launch_status();
+    return launch_quantize(x, rows, cols, q, s, stream);
 }
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -445,12 +480,7 @@ w8a8_status_t w8a8_linear_noalloc(const w8a8_bf16_t *x, int64_t M, int64_t K,
     int8_t *xq = static_cast<int8_t *>(scratch);
     float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + kNoAllocCodeBytes);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t KB = K / 128;
-    const int64_t nblocks = (M / 128) * KB;
-    const int64_t grid = std::min<int64_t>(nblocks, static_cast<int64_t>(g_dev[dev].sms) * 8);
-    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kThreads, 0, st>>>(
-        x, K, nblocks, KB, xq, xs);
-    W8A8_TRY(launch_status());
+    W8A8_TRY(launch_quantize(x, M, K, xq, xs, st));
     W8A8_TRY(gemm_i8_impl(xq, xs, M, K, w, bias, y, st));
     if (path_taken != nullptr)
         *path_taken = W8A8_PATH_INT8;
