@@ -54,7 +54,8 @@ def load(path=None):
         lib = ctypes.CDLL(build())
     for name in ["oracle_block_quantize", "oracle_block_sums", "oracle_w8a8_linear",
                  "oracle_w8a8_linear_at", "oracle_rmsnorm", "oracle_rmsnorm_apply",
-                 "oracle_bf16_linear", "oracle_bf16_linear_at", "oracle_num_threads"]:
+                 "oracle_bf16_linear", "oracle_bf16_linear_at", "oracle_num_threads",
+                 "oracle_row_quantize", "oracle_row_linear", "oracle_row_linear_at"]:
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_f32_to_bf16.restype = None
     if path is None:
@@ -119,6 +120,41 @@ class Oracle:
                                             _i64(ms.size), _ptr(out))
         if rc:
             raise ValueError("w8a8_linear_at: bad arguments")
+        return out
+
+    # -- per-row / per-output-channel operator (TurboT2VA paper, W8A8 paragraph) --------
+    def row_quantize(self, x_bits):
+        """Codes and one FP32 scale per row (activation rows or weight output channels)."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        r, c = x.shape
+        q = np.empty((r, c), dtype=np.int8)
+        s = np.empty(r, dtype=np.float32)
+        if self.lib.oracle_row_quantize(_ptr(x), _i64(r), _i64(c), _ptr(q), _ptr(s)):
+            raise ValueError("row_quantize: bad arguments")
+        return q, s
+
+    def row_linear(self, xq, xs, wq, ws, bias=None, m0=0, rows=None):
+        xq, xs, wq, ws, bias = _prep(xq, xs, wq, ws, bias)
+        M, K = xq.shape
+        N = wq.shape[0]
+        rows = M - m0 if rows is None else rows
+        out = np.empty((rows, N), dtype=np.float32)
+        if self.lib.oracle_row_linear(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(bias),
+                                      _i64(M), _i64(K), _i64(N), _i64(m0), _i64(rows),
+                                      _ptr(out)):
+            raise ValueError("row_linear: bad arguments")
+        return out
+
+    def row_linear_at(self, xq, xs, wq, ws, bias, ms, ns):
+        xq, xs, wq, ws, bias = _prep(xq, xs, wq, ws, bias)
+        ms = np.ascontiguousarray(ms, dtype=np.int64)
+        ns = np.ascontiguousarray(ns, dtype=np.int64)
+        out = np.empty(ms.size, dtype=np.float32)
+        if self.lib.oracle_row_linear_at(_ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(bias),
+                                         _i64(xq.shape[0]), _i64(xq.shape[1]),
+                                         _i64(wq.shape[0]), _ptr(ms), _ptr(ns), _i64(ms.size),
+                                         _ptr(out)):
+            raise ValueError("row_linear_at: bad arguments")
         return out
 
     # -- RMSNorm (TurboDiffusion article, inference list item 5) -----------------------

@@ -24,6 +24,8 @@
  *     paragraph.
  *   - BF16 fallback linear with the retained BF16 weight: TurboT2VA paper,
  *     inference-stack section, guard paragraph.
+ *   - The per-row / per-output-channel post-scale operator (the paper's own W8A8
+ *     kernel): TurboT2VA paper, W8A8 operator paragraph (see the per-row section).
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   rounding of x/s to an integer is round-half-to-even; x/s is one IEEE FP32 division
@@ -190,6 +192,82 @@ int oracle_w8a8_linear_at(const int8_t *xq, const float *xs, const int8_t *wq, c
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < count; ++t)
         out[t] = w8a8_output(xq, xs, wq, ws, bias, K, ms[t], ns[t]);
+    return 0;
+}
+
+/* ---------------------------------------------------------------- per-row W8A8 ----- */
+/* The post-scale W8A8 operator of the TurboT2VA paper (inference-stack section, W8A8
+ * operator paragraph): dynamic per-row activation scales and static per-output-channel
+ * weight scales s = max(||row||_inf, eps) / 127 with eps = 1e-4, INT8 codes per row,
+ * INT8 products accumulated in INT32 over the whole of K, then both scales and the bias
+ * applied once.  The page's formula itself did not survive extraction; the readings are:
+ * eps is the FP32 value nearest 1e-4, the codes follow the block path's rule (IEEE FP32
+ * quotient by the stored scale, half-to-even, clamp to [-127, 127]), and the output is
+ * fl(fl(float(acc) * fl(sx * sw)) + b), float(acc) being the INT32 sum rounded to FP32. */
+#define ROW_EPS 1e-4f
+
+/* x: [rows, cols] BF16 -> q: [rows, cols] INT8 codes, s: [rows] FP32 scales. */
+int oracle_row_quantize(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s)
+{
+    if (rows < 0 || cols < 0)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float absmax = 0.0f;
+        for (int64_t j = 0; j < cols; ++j) {
+            const float a = fabsf(bf16_to_f32(x[r * cols + j]));
+            if (a > absmax)
+                absmax = a;
+        }
+        const float sc = (absmax > ROW_EPS ? absmax : ROW_EPS) / 127.0f;
+        s[r] = sc;
+        for (int64_t j = 0; j < cols; ++j)
+            q[r * cols + j] = quantize_one(bf16_to_f32(x[r * cols + j]), sc);
+    }
+    return 0;
+}
+
+/* One output element of the per-row operator. */
+static float row_output(const int8_t *xq, const float *xs, const int8_t *wq, const float *ws,
+                        const uint16_t *bias, int64_t K, int64_t m, int64_t n)
+{
+    int64_t acc = 0;
+    for (int64_t k = 0; k < K; ++k)
+        acc += (int64_t)xq[m * K + k] * (int64_t)wq[n * K + k];
+    const float scale = xs[m] * ws[n];
+    const float v = (float)(int32_t)acc * scale;
+    const float b = bias ? bf16_to_f32(bias[n]) : 0.0f;
+    return v + b;
+}
+
+/* Rows [m0, m0 + rows) of the FP32 output: out[(m - m0) * N + n].  K < 2^31 / 127^2 keeps
+ * every sum inside INT32. */
+int oracle_row_linear(const int8_t *xq, const float *xs, const int8_t *wq, const float *ws,
+                      const uint16_t *bias, int64_t M, int64_t K, int64_t N, int64_t m0,
+                      int64_t rows, float *out)
+{
+    if (M < 0 || K < 0 || N < 0 || K > 133000 || m0 < 0 || rows < 0 || m0 + rows > M)
+        return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t n = 0; n < N; ++n)
+            out[i * N + n] = row_output(xq, xs, wq, ws, bias, K, m0 + i, n);
+    return 0;
+}
+
+/* The FP32 output at count sampled coordinates (ms[t], ns[t]). */
+int oracle_row_linear_at(const int8_t *xq, const float *xs, const int8_t *wq, const float *ws,
+                         const uint16_t *bias, int64_t M, int64_t K, int64_t N, const int64_t *ms,
+                         const int64_t *ns, int64_t count, float *out)
+{
+    if (M < 0 || K < 0 || N < 0 || K > 133000)
+        return -1;
+    for (int64_t t = 0; t < count; ++t)
+        if (ms[t] < 0 || ms[t] >= M || ns[t] < 0 || ns[t] >= N)
+            return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < count; ++t)
+        out[t] = row_output(xq, xs, wq, ws, bias, K, ms[t], ns[t]);
     return 0;
 }
 

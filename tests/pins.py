@@ -406,4 +406,121 @@ def pin_bf16_textbook(o):
                                   y[ms, ns].astype(np.float32))
 
 
+# ---------------------------------------------------------------- per-row operator
+# TurboT2VA paper, W8A8 operator paragraph: s = max(||row||_inf, 1e-4) / 127 per activation
+# row and per weight output channel, INT32 accumulation over all of K, both scales and the
+# bias once.
+
+ROW_EPS32 = np.float32(1e-4)
+
+
+def pin_row_scale_closed_forms(o):
+    """Rows whose absmax is 127 * 2^e get s = 2^e; an all-zero row and a row below the
+    floor get the floor's scale fl(1e-4 / 127); the floor row's largest code is the
+    correctly rounded quotient (well below 127)."""
+    es = [-20, -6, 0, 3, 11]
+    K = 200
+    x = np.zeros((len(es) + 2, K))
+    for i, e in enumerate(es):
+        x[i, 7] = -127.0 * 2.0 ** e
+        x[i, 8:] = _rng(i).uniform(-1, 1, K - 8) * 2.0 ** e * 100
+    x[len(es) + 1, 3] = 2.0 ** -15          # below the 1e-4 floor
+    q, s = o.row_quantize(_bf16(x))
+    for i, e in enumerate(es):
+        assert s[i] == np.float32(2.0 ** e), (i, s[i])
+        assert q[i, 7] == -127
+    floor = _div_f32(ROW_EPS32, np.float32(127))
+    assert s[len(es)] == floor and s[len(es) + 1] == floor
+    assert not q[len(es)].any()
+    expect = int(np.rint(_div_f32(np.float32(2.0 ** -15), floor)))
+    assert q[len(es) + 1, 3] == expect and 0 < expect < 127, expect
+
+
+def pin_row_grid_roundtrip(o):
+    """Inputs c * 2^e with integer |c| <= 127 and some |c| = 127 per row: codes are c."""
+    r = _rng(31)
+    M, K = 9, 300
+    c = r.integers(-127, 128, (M, K))
+    c[np.arange(M), r.integers(0, K, M)] = 127 * r.choice([-1, 1], M)
+    e = r.integers(-19, 30, M)          # 127 * 2^e stays above the 1e-4 floor
+    q, s = o.row_quantize(_bf16(c * 2.0 ** e[:, None]))
+    np.testing.assert_array_equal(q.astype(np.int64), c)
+    np.testing.assert_array_equal(s, (2.0 ** e).astype(np.float32))
+
+
+def pin_row_error_bound(o):
+    """|x - q s| <= s (1/2 + 2^-17) for rows above the floor; each row's absmax element
+    maps to +-127; codes never leave [-127, 127]."""
+    r = _rng(32)
+    x = r.standard_t(3, (40, 257)) * np.exp(r.uniform(-8, 8, (40, 1)))
+    bits = _bf16(x)
+    q, s = o.row_quantize(bits)
+    xf = _f32(bits)
+    sd = s.astype(np.float64)[:, None]
+    assert np.all(np.abs(xf - q * sd) <= sd * (0.5 + 2.0 ** -17))
+    am = np.argmax(np.abs(xf), axis=1)
+    assert np.all(np.abs(q[np.arange(40), am]) == 127)
+    assert q.min() >= -127
+
+
+def pin_row_linear_bruteforce(o):
+    """Against a float64 dequantize-then-GEMM on odd shapes, with per-row and per-column
+    scales that differ by up to 2^24 (a transposed or swapped scale index fails), within
+    the four FP32 roundings of the epilogue."""
+    r = _rng(33)
+    M, K, N = 6, 333, 9
+    xb = _bf16(r.standard_normal((M, K)) * 2.0 ** r.integers(-12, 12, (M, 1)))
+    wb = _bf16(r.standard_normal((N, K)) * 2.0 ** r.integers(-12, 12, (N, 1)))
+    bb = _bf16(r.standard_normal(N) * 0.1)
+    xq, xs = o.row_quantize(xb)
+    wq, ws = o.row_quantize(wb)
+    out = o.row_linear(xq, xs, wq, ws, bb).astype(np.float64)
+    acc = xq.astype(np.int64) @ wq.astype(np.int64).T
+    main = acc * xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :]
+    ref = main + _f32(bb)[None, :]
+    assert np.all(np.abs(out - ref) <= 2.0 ** -22 * (np.abs(main) + np.abs(ref)) + 1e-30)
+    # sampled entry point agrees bit for bit
+    ms, ns = np.array([0, 5, 3]), np.array([8, 0, 4])
+    np.testing.assert_array_equal(o.row_linear_at(xq, xs, wq, ws, bb, ms, ns),
+                                  out[ms, ns].astype(np.float32))
+
+
+def pin_row_int32_to_fp32(o):
+    """INT32 sums of 2^24 + 1 and 2^24 + 3 are rounded to FP32 (half to even: 2^24 and
+    2^24 + 4) before the scales multiply them.  With unit scales that is the whole
+    output; with the weight scale fl(128 / 127) the output is fl(fl(sum) * scale), which
+    differs from rounding the exact product once."""
+    K = 1042
+    differs = []
+    for w_absmax in (127.0, 128.0):
+        w = np.zeros((1, K))
+        w[0, :1040] = w_absmax
+        w[0, 1040] = 24.25 if w_absmax == 128.0 else 24.0
+        w[0, 1041] = 1
+        for extra, sum_f32 in ((9, 2.0 ** 24), (11, 2.0 ** 24 + 4)):
+            x = np.zeros((1, K))
+            x[0, :1041] = 127
+            x[0, 1041] = extra
+            xq, xs = o.row_quantize(_bf16(x))
+            wq, ws = o.row_quantize(_bf16(w))
+            acc = int(xq.astype(np.int64) @ wq.astype(np.int64).T)
+            assert xs[0] == 1 and acc == 2 ** 24 + extra - 8, (xs, acc)
+            scale = np.float32(xs[0]) * np.float32(ws[0])
+            expect = np.float32(np.float32(sum_f32) * scale)
+            got = o.row_linear(xq, xs, wq, ws, None)[0, 0]
+            assert got == expect, (w_absmax, extra, got, expect)
+            if w_absmax == 128.0:
+                differs.append(expect != np.float32(np.float64(acc) * np.float64(scale)))
+    assert any(differs)     # the case separates the two rounding orders
+
+
+def pin_row_bias_once(o):
+    """All-zero codes: the output is the bias, added once."""
+    xq = np.zeros((3, 256), np.int8)
+    wq = np.zeros((5, 256), np.int8)
+    bb = _bf16(np.array([1.5, -2.25, 0.0, 7.0, -0.125]))
+    out = o.row_linear(xq, np.ones(3, np.float32), wq, np.ones(5, np.float32), bb)
+    np.testing.assert_array_equal(out, np.tile(_f32(bb).astype(np.float32), (3, 1)))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

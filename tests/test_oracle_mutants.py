@@ -48,6 +48,18 @@ MUTANTS = [
     ("fallback_w_reversed_k", "(double)bf16_to_f32(w[n * K + k]);",
      "(double)bf16_to_f32(w[n * K + (K - 1 - k)]);"),
     ("fallback_drop_bias", "return (float)acc + b;", "return (float)acc;"),
+    ("row_floor_on_scale", "const float sc = (absmax > ROW_EPS ? absmax : ROW_EPS) / 127.0f;",
+     "const float sc = (absmax / 127.0f > ROW_EPS ? absmax / 127.0f : ROW_EPS);"),
+    ("row_floor_1e-3", "#define ROW_EPS 1e-4f", "#define ROW_EPS 1e-3f"),
+    ("row_no_abs", "const float a = fabsf(bf16_to_f32(x[r * cols + j]));",
+     "const float a = bf16_to_f32(x[r * cols + j]);"),
+    ("row_drop_weight_scale", "const float scale = xs[m] * ws[n];",
+     "const float scale = xs[m];"),
+    ("row_weight_scale_halved_index", "const float scale = xs[m] * ws[n];",
+     "const float scale = xs[m] * ws[n / 2];"),
+    ("row_sum_in_double", "const float v = (float)(int32_t)acc * scale;",
+     "const float v = (float)((double)acc * (double)scale);"),
+    ("row_bias_twice", "return v + b;", "return v + b + b;"),
 ]
 # commuted_product_noop rewrites without changing the arithmetic (FP32 multiplication
 # commutes): it checks that the harness does not report every rewrite as caught.
