@@ -55,6 +55,11 @@ _SIGS = {
     "w8a8_debug_block_sums": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                               ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p],
     "w8a8_debug_wait_timeout": [ctypes.c_uint64, ctypes.c_void_p],
+    "w8a8_rowwise_quantize": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                              ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_rowwise_linear": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                            ctypes.c_void_p, ctypes.c_void_p],
 }
 
 
@@ -130,6 +135,39 @@ def quantize_weight(w):
     _check("w8a8_quantize_weight", lib().w8a8_quantize_weight(_ptr(w), N, K, _ptr(wq), _ptr(ws),
                                                                _stream(w.device)))
     return wq, ws
+
+
+def rowwise_quantize(x, q=None, s=None):
+    """Per-row INT8 quantization of a BF16 [rows, K] matrix (TurboT2VA's post-scale
+    operator: s = max(||row||_inf, 1e-4) / 127) -> (q int8 [rows, K], s float32 [rows]).
+    For a weight [N, K] this gives its per-output-channel codes and scales."""
+    _need(x, torch.bfloat16, "x")
+    rows, K = x.shape
+    q = torch.empty((rows, K), dtype=torch.int8, device=x.device) if q is None else q
+    s = torch.empty((rows,), dtype=torch.float32, device=x.device) if s is None else s
+    _check("w8a8_rowwise_quantize", lib().w8a8_rowwise_quantize(_ptr(x), rows, K, _ptr(q), _ptr(s),
+                                                                 _stream(x.device)))
+    return q, s
+
+
+def rowwise_linear_prequant(xq, xs, wq, ws, bias=None, out=None):
+    """y = bf16(float(xq wq^T) * (xs[m] ws[n]) + bias) with INT32 accumulation over all of K."""
+    _need(xq, torch.int8, "xq")
+    _need(wq, torch.int8, "wq")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _check("w8a8_rowwise_linear", lib().w8a8_rowwise_linear(
+        _ptr(xq), _ptr(xs), M, K, _ptr(wq), _ptr(ws), N, _ptr(bias), _ptr(y), _stream(xq.device)))
+    return y
+
+
+def rowwise_linear(x, wq, ws, bias=None, out=None):
+    """The per-row operator on BF16 activations: per-row quantization, then the GEMM."""
+    xq, xs = rowwise_quantize(x)
+    return rowwise_linear_prequant(xq, xs, wq, ws, bias, out)
 
 
 def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):

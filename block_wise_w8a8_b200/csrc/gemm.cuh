@@ -11,6 +11,9 @@
 //   kI8Dump   : same main loop; the epilogue writes P[m,n,kb] itself (test hook).
 //   kBf16     : BF16 x BF16 -> FP32 GEMM (kind::f16) for the guard's fallback (TurboT2VA
 //               paper, guard paragraph), FP32 accumulation over all of K in tensor memory.
+//   kI8Row    : the per-row / per-output-channel post-scale W8A8 operator (TurboT2VA
+//               paper, W8A8 operator paragraph): INT8 x INT8 accumulated in INT32 over all
+//               of K in tensor memory, both scales and the bias applied once per tile.
 //
 // Tile 128 x 256 (BM x BN), one 128-byte K slice per pipeline stage (128 INT8 or 64 BF16
 // elements = exactly one K block of the INT8 path), 4 stages of 48 KB in shared memory,
@@ -38,7 +41,7 @@
 namespace w8a8 {
 namespace gemm {
 
-enum class Mode : int { kI8Scaled = 0, kI8Dump = 1, kBf16 = 2 };
+enum class Mode : int { kI8Scaled = 0, kI8Dump = 1, kBf16 = 2, kI8Row = 3 };
 
 constexpr int BM = 128;
 constexpr int BN = 256;
@@ -134,7 +137,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p)
 {
-    constexpr bool kInt8 = (kMode != Mode::kBf16);
+    constexpr bool kInt8 = (kMode != Mode::kBf16);                    // INT8 operands
+    constexpr bool kPerKb = (kMode == Mode::kI8Scaled || kMode == Mode::kI8Dump);   // per-K-block sums
     constexpr int kSliceElems = kInt8 ? 128 : 64;
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bool ok = true;
             for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
                 uint32_t buf = acc_i & 1;
-                if (!kInt8) {
+                if (!kPerKb) {
                     if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
                         ok = false;
                         break;
@@ -214,7 +218,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 for (int ks = 0; ks < p.kslices; ++ks, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    if (kInt8) {
+                    if (kPerKb) {
                         buf = acc_i & 1;
                         if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
                             ok = false;
@@ -232,18 +236,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         // each MMA consumes 32 bytes of K: advance start address by 32 B
-                        if (kInt8)
+                        if (kPerKb)
                             umma_i8(d, ad + 2 * k, bd + 2 * k, idesc, 1u);
+                        else if (kInt8)
+                            umma_i8(d, ad + 2 * k, bd + 2 * k, idesc, (ks | k) != 0);
                         else
                             umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (ks | k) != 0);
                     }
                     umma_commit(&sm.empty[s]);
-                    if (kInt8) {
+                    if (kPerKb) {
                         umma_commit(&sm.tfull[buf]);
                         ++acc_i;
                     }
                 }
-                if (!kInt8 && ok) {
+                if (!kPerKb && ok) {
                     umma_commit(&sm.tfull[buf]);
                     ++acc_i;
                 }
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             fill[i] = kAccInit;
-        if (kInt8) {
+        if (kPerKb) {
 #pragma unroll
             for (int b = 0; b < 2; ++b)
 #pragma unroll
@@ -421,6 +427,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 if (!ok)
                     break;
+            }
+        } else if (kMode == Mode::kI8Row) {
+            // Per-row / per-output-channel scales (TurboT2VA paper, W8A8 operator
+            // paragraph): one INT32 accumulator per tile over all of K, read once;
+            // y = bf16(fl(fl(float(acc) * fl(xs[m] * ws[n])) + b)), no fused multiply-add.
+            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+                const uint32_t buf = acc_i & 1;
+                if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
+                    break;
+                tc_fence_after();
+                const int64_t m = static_cast<int64_t>(tm) * BM + row;
+                const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                const uint32_t tb = lane_base + buf * BN;
+                const float sx = p.xs[m];
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tb + c * 32, r);
+                    tmem_wait_ld();
+                    const int64_t nc = n0 + c * 32;
+                    if (nc < p.N) {
+                        uint16_t *dst = p.y + m * p.N + nc;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.ws + nc + g * 8));
+                            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.ws + nc + g * 8 + 4));
+                            const float wsv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                            float bb[8];
+                            if (p.bias != nullptr) {
+                                const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + nc + g * 8));
+                                bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
+                                bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
+                                bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
+                                bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    bb[i] = 0.0f;
+                            }
+                            float v[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float a = __int2float_rn(static_cast<int>(r[g * 8 + i]));
+                                v[i] = __fadd_rn(__fmul_rn(a, __fmul_rn(sx, wsv[i])), bb[i]);
+                            }
+                            uint4 o;
+                            o.x = pack_bf16x2(v[0], v[1]);
+                            o.y = pack_bf16x2(v[2], v[3]);
+                            o.z = pack_bf16x2(v[4], v[5]);
+                            o.w = pack_bf16x2(v[6], v[7]);
+                            *reinterpret_cast<uint4 *>(dst + g * 8) = o;
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.tempty[buf]);
+                ++acc_i;
             }
         } else {
             // BF16: one accumulator per tile, read once at the end of the tile.

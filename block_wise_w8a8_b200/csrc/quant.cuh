@@ -315,6 +315,58 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ per-row quantizer --
+// x [rows, K] BF16 -> q [rows, K] INT8, s [rows] FP32 with s = max(||row||_inf, 1e-4) / 127
+// (TurboT2VA paper, W8A8 operator paragraph: dynamic per-row activation scales, static
+// per-output-channel weight scales; eps = the FP32 value nearest 1e-4).  One warp per row:
+// pass 1 reads the row with 16-byte loads for its absmax (warp shuffles), pass 2 reads it
+// again (now from L1 / L2) for the codes, written with 8-byte stores.  Values within 2^-14
+// of a half-integer are re-coded with the IEEE division, as in quantize_blocks_kernel.
+constexpr float kRowEps = 1e-4f;
+constexpr int kRowWarps = 8;
+
+__global__ void __launch_bounds__(kRowWarps * 32)
+    row_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows, int64_t K,
+                        int8_t *__restrict__ q, float *__restrict__ s)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunks = K / 8;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5); r < rows;
+         r += static_cast<int64_t>(gridDim.x) * kRowWarps) {
+        const uint16_t *xr = x + r * K;
+        uint32_t m2 = 0;
+#pragma unroll 4
+        for (int64_t c = lane; c < nchunks; c += 32) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c * 8));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            m2 = absmax8_bits(w, m2);
+        }
+        uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        const float amax = __uint_as_float(m << 16);
+        const float sc = __fdiv_rn(fmaxf(amax, kRowEps), 127.0f);
+        const float rc = __frcp_rn(sc);     // sc >= 1e-4 / 127: no overflow
+        if (lane == 0)
+            s[r] = sc;
+        int8_t *qr = q + r * K;
+#pragma unroll 4
+        for (int64_t c = lane; c < nchunks; c += 32) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c * 8));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t band;
+            *reinterpret_cast<uint2 *>(qr + c * 8) = quantize8_fast(w, rc, band);
+            while (band != 0) {
+                const int e = __ffs(band) - 1;
+                band &= band - 1;
+                const float v1 = __uint_as_float(static_cast<uint32_t>(xr[c * 8 + e]) << 16);
+                qr[c * 8 + e] = static_cast<int8_t>(code_exact(v1, sc));
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ fused RMSNorm ------
 
 constexpr int kNormCluster = 8;    // CTAs sharing one 128-row strip

@@ -19,11 +19,13 @@ using namespace w8a8;
 constexpr int kMaxDevices = 64;
 // TMA coordinates are signed 32-bit: matrix extents stay below 2^31.
 constexpr int64_t kMaxTmaCoord = (int64_t{1} << 31) - 128;
+// Per-row operator: K * 127^2 must stay inside INT32 (the accumulator holds all of K).
+constexpr int64_t kRowMaxK = 133120;
 
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
-    bool gemm_attr_set[3] = {false, false, false};
+    bool gemm_attr_set[4] = {false, false, false, false};
     bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -528,6 +530,60 @@ w8a8_status_t w8a8_bf16_linear(const w8a8_bf16_t *x, const w8a8_bf16_t *w,
     if (bias != nullptr)
         W8A8_TRY(check_device_ptr(bias));
     return bf16_impl(x, w, bias, y, M, K, N, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_rowwise_quantize(const w8a8_bf16_t *x, int64_t rows, int64_t K, int8_t *q,
+                                    float *s, void *stream)
+{
+    if (rows < 0 || K < 0)
+        return W8A8_ERR_INVALID_ARG;
+    if (K % 8)
+        return W8A8_ERR_SHAPE;
+    if (rows == 0 || K == 0)
+        return rows == 0 ? W8A8_OK : W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(x));
+    W8A8_TRY(check_device_ptr(q));
+    W8A8_TRY(check_device_ptr(s));
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u))
+        return W8A8_ERR_ALIGNMENT;
+    int dev;
+    W8A8_TRY(current_device(dev));
+    const int64_t blocks = (rows + quant::kRowWarps - 1) / quant::kRowWarps;
+    const int64_t grid = std::min<int64_t>(blocks, static_cast<int64_t>(g_dev[dev].sms) * 16);
+    quant::row_quantize_kernel<<<static_cast<unsigned>(grid), quant::kRowWarps * 32, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(x, rows, K, q, s);
+    return launch_status();
+}
+
+w8a8_status_t w8a8_rowwise_linear(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                                  const int8_t *wq, const float *ws, int64_t N,
+                                  const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *stream)
+{
+    if (M < 0 || K < 0 || N < 0)
+        return W8A8_ERR_INVALID_ARG;
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    if (K == 0 || M % 128 || K % 128 || N % 128 || K > kRowMaxK)
+        return W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(xs));
+    W8A8_TRY(check_device_ptr(wq));
+    W8A8_TRY(check_device_ptr(ws));
+    W8A8_TRY(check_device_ptr(y));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(ws) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(xs) & 3u) || (bias != nullptr && !aligned16(bias)))
+        return W8A8_ERR_ALIGNMENT;
+    gemm::Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.xs = xs;
+    p.ws = ws;
+    p.bias = bias;
+    p.y = y;
+    return launch_gemm<gemm::Mode::kI8Row>(xq, wq, p, static_cast<cudaStream_t>(stream));
 }
 
 w8a8_status_t w8a8_debug_block_sums(const int8_t *xq, const int8_t *wq, int64_t M, int64_t K,

@@ -185,6 +185,33 @@ W8A8_API w8a8_status_t w8a8_bf16_linear(const w8a8_bf16_t *x, const w8a8_bf16_t 
                                const w8a8_bf16_t *bias, w8a8_bf16_t *y, int64_t M, int64_t K,
                                int64_t N, void *stream);
 
+/* ---- The per-row / per-output-channel post-scale operator ---------------------------
+ * TurboT2VA paper, inference-stack section, W8A8 operator paragraph: activations get one
+ * scale per row (dynamic) and weights one per output channel (static),
+ *   s = max(||row||_inf, eps) / 127,  eps = 1e-4 (as the FP32 value nearest it),
+ * codes q = clamp(round_half_even(fl32(v / s)), -127, 127) as in the block-wise path,
+ * INT8 products accumulated in INT32 over the whole of K, and both scales and the bias
+ * applied once: y[m,n] = bf16( fl(fl(float(acc[m,n]) * fl(xs[m] * ws[n])) + bias[n]) ),
+ * float(acc) being the INT32 sum rounded to FP32.  (The page's formula itself was lost in
+ * extraction; these are the readings the oracle and the kernels share.) */
+
+/* Per-row quantization of x [rows, K] BF16 (activations, or a weight [N, K] for its
+ * per-output-channel codes): q [rows, K] INT8 and s [rows] FP32, caller-owned device
+ * buffers; x and q 16-byte aligned, s 4-byte aligned.  K a multiple of 8 and > 0 (else
+ * W8A8_ERR_SHAPE).  Asynchronous on `stream`. */
+W8A8_API w8a8_status_t w8a8_rowwise_quantize(const w8a8_bf16_t *x, int64_t rows, int64_t K,
+                                             int8_t *q, float *s, void *stream);
+
+/* y [M, N] BF16 from xq [M, K] / xs [M] (per-row) and wq [N, K] / ws [N] (per output
+ * channel), bias [N] BF16 or NULL.  M, K, N multiples of 128 and K <= 133120 (so every
+ * INT32 sum fits), else W8A8_ERR_SHAPE; xq, wq, ws, y, bias 16-byte aligned, xs 4-byte
+ * aligned, else W8A8_ERR_ALIGNMENT.  The INT8 tcgen05 main loop of w8a8_linear with one
+ * accumulator per 128 x 256 tile over all of K.  Asynchronous on `stream`. */
+W8A8_API w8a8_status_t w8a8_rowwise_linear(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                                           const int8_t *wq, const float *ws, int64_t N,
+                                           const w8a8_bf16_t *bias, w8a8_bf16_t *y,
+                                           void *stream);
+
 /* Test hook: the INT32 partial products P[m, n, kb] of the INT8 GEMM, written by the
  * same tensor-core main loop as w8a8_linear, for xq [M, K] and wq [N, K] (M, K, N
  * multiples of 128).  out: [M, N, K/128] INT32 device buffer. */
