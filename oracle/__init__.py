@@ -55,7 +55,8 @@ def load(path=None):
     for name in ["oracle_block_quantize", "oracle_block_sums", "oracle_w8a8_linear",
                  "oracle_w8a8_linear_at", "oracle_rmsnorm", "oracle_rmsnorm_apply",
                  "oracle_bf16_linear", "oracle_bf16_linear_at", "oracle_num_threads",
-                 "oracle_row_quantize", "oracle_row_linear", "oracle_row_linear_at"]:
+                 "oracle_row_quantize", "oracle_row_linear", "oracle_row_linear_at",
+                 "oracle_mod_rmsnorm", "oracle_gated_residual"]:
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_f32_to_bf16.restype = None
     if path is None:
@@ -182,6 +183,50 @@ class Oracle:
         if rc:
             raise ValueError("rmsnorm_apply: bad arguments")
         return y
+
+    # -- modulated RMSNorm and gated residual (TurboT2VA paper, fused-operator paragraph)
+    def mod_rmsnorm(self, x_bits, gamma_bits, scale_bits, shift_bits, T, eps, m0=0, rows=None):
+        """y = bf16(fl(fl(n * fl(1 + scale[m / T])) + shift[m / T])), n = x * rstd (times
+        gamma when given); scale and shift [M / T, K]."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        g = None if gamma_bits is None else np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+        sc = np.ascontiguousarray(scale_bits, dtype=np.uint16)
+        sh = np.ascontiguousarray(shift_bits, dtype=np.uint16)
+        M, K = x.shape
+        if T <= 0 or M % T or sc.shape != (M // T, K) or sh.shape != (M // T, K) or \
+                (g is not None and g.shape != (K,)):
+            raise ValueError("mod_rmsnorm: bad shapes")
+        rows = M - m0 if rows is None else rows
+        y = np.empty((rows, K), dtype=np.uint16)
+        rstd = np.empty(rows, dtype=np.float32)
+        rc = self.lib.oracle_mod_rmsnorm(_ptr(x), _ptr(g), _ptr(sc), _ptr(sh), _i64(T),
+                                         ctypes.c_float(eps), _i64(M), _i64(K), _i64(m0),
+                                         _i64(rows), _ptr(y), _ptr(rstd))
+        if rc:
+            raise ValueError("mod_rmsnorm: bad arguments")
+        return y, rstd
+
+    def gated_residual(self, v, r_bits, gate_bits, T, M, ms=None, ns=None):
+        """out = bf16(fl(r + fl(gate[m / T, n] * v))).  With ms, ns: v and r_bits hold the
+        values at those points; without: v and r_bits are the full [M, N] arrays."""
+        g = np.ascontiguousarray(gate_bits, dtype=np.uint16)
+        N = g.shape[1]
+        if ms is None:
+            shape = np.shape(v)
+            ms, ns = np.indices(shape).reshape(2, -1)
+        else:
+            shape = np.shape(ms)
+        v = np.ascontiguousarray(v, dtype=np.float32).reshape(-1)
+        r = np.ascontiguousarray(r_bits, dtype=np.uint16).reshape(-1)
+        ms = np.ascontiguousarray(ms, dtype=np.int64).reshape(-1)
+        ns = np.ascontiguousarray(ns, dtype=np.int64).reshape(-1)
+        if T <= 0 or M % T or g.shape[0] != M // T or not (v.size == r.size == ms.size == ns.size):
+            raise ValueError("gated_residual: bad shapes")
+        out = np.empty(ms.size, dtype=np.uint16)
+        if self.lib.oracle_gated_residual(_ptr(v), _ptr(r), _ptr(g), _i64(T), _i64(M), _i64(N),
+                                          _ptr(ms), _ptr(ns), _i64(ms.size), _ptr(out)):
+            raise ValueError("gated_residual: bad arguments")
+        return out.reshape(shape)
 
     # -- BF16 fallback (TurboT2VA paper, guard paragraph) ------------------------------
     def bf16_linear(self, x_bits, w_bits, bias=None, m0=0, rows=None):

@@ -320,6 +320,70 @@ int oracle_rmsnorm_apply(const uint16_t *x, const uint16_t *gamma, const float *
     return 0;
 }
 
+/* ------------------------------------------- modulated RMSNorm, gated residual ----- */
+/* TurboT2VA paper, fused-operator paragraph: normalization combined with modality- and
+ * timestep-dependent modulation (modulated RMS normalization, adaptive scale-shift
+ * modulation), and gated residual updates.  The page names these operations without
+ * formulas; the readings are the adaptive-norm form of diffusion transformers, each
+ * group of T consecutive rows (one sample's tokens) sharing one modulation row:
+ *   modulated RMSNorm: n = fl(x * rstd), times gamma[k] when gamma is given (FP32
+ *     product), then y = bf16( fl( fl(n * fl(1 + scale[b, k])) + shift[b, k] ) ) with
+ *     b = m / T; rstd as for the plain RMSNorm; no intermediate BF16 rounding.
+ *   gated residual: out = bf16( fl( r[m, n] + fl(gate[b, n] * v[m, n]) ) ), v the FP32
+ *     linear output (bias included) that the plain linear would round to BF16, b = m / T.
+ */
+static void row_apply_mod(const uint16_t *xrow, const uint16_t *gamma, const uint16_t *scale,
+                          const uint16_t *shift, float rstd, int64_t K, uint16_t *yrow)
+{
+    for (int64_t k = 0; k < K; ++k) {
+        float n = bf16_to_f32(xrow[k]) * rstd;
+        if (gamma)
+            n = n * bf16_to_f32(gamma[k]);
+        const float a = 1.0f + bf16_to_f32(scale[k]);
+        const float u = n * a;
+        yrow[k] = f32_to_bf16(u + bf16_to_f32(shift[k]));
+    }
+}
+
+/* Rows [m0, m0 + rows) of the modulated RMSNorm: x [M, K], gamma [K] or NULL, scale and
+ * shift [M / T, K]; y [rows, K] BF16 bits, rstd [rows]. */
+int oracle_mod_rmsnorm(const uint16_t *x, const uint16_t *gamma, const uint16_t *scale,
+                       const uint16_t *shift, int64_t T, float eps, int64_t M, int64_t K,
+                       int64_t m0, int64_t rows, uint16_t *y, float *rstd)
+{
+    if (K <= 0 || T <= 0 || M % T != 0 || m0 < 0 || rows < 0 || m0 + rows > M)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < rows; ++i) {
+        const int64_t m = m0 + i;
+        const int64_t b = m / T;
+        const float r = row_rstd(x + m * K, K, eps);
+        rstd[i] = r;
+        row_apply_mod(x + m * K, gamma, scale + b * K, shift + b * K, r, K, y + i * K);
+    }
+    return 0;
+}
+
+/* The gated residual at S points (ms[t], ns[t]) of an [M, N] output: v[t] the FP32 linear
+ * output there, r[t] the residual's BF16 bits there, gate [M / T, N]; out[t] BF16 bits. */
+int oracle_gated_residual(const float *v, const uint16_t *r, const uint16_t *gate, int64_t T,
+                          int64_t M, int64_t N, const int64_t *ms, const int64_t *ns, int64_t S,
+                          uint16_t *out)
+{
+    if (T <= 0 || M % T != 0 || N <= 0 || S < 0)
+        return -1;
+    for (int64_t t = 0; t < S; ++t)
+        if (ms[t] < 0 || ms[t] >= M || ns[t] < 0 || ns[t] >= N)
+            return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < S; ++t) {
+        const int64_t b = ms[t] / T;
+        const float gv = bf16_to_f32(gate[b * N + ns[t]]) * v[t];
+        out[t] = f32_to_bf16(bf16_to_f32(r[t]) + gv);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- BF16 linear ------ */
 
 static float bf16_output(const uint16_t *x, const uint16_t *w, const uint16_t *bias,

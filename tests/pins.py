@@ -503,7 +503,7 @@ def pin_row_int32_to_fp32(o):
             x[0, 1041] = extra
             xq, xs = o.row_quantize(_bf16(x))
             wq, ws = o.row_quantize(_bf16(w))
-            acc = int(xq.astype(np.int64) @ wq.astype(np.int64).T)
+            acc = int((xq.astype(np.int64) @ wq.astype(np.int64).T)[0, 0])
             assert xs[0] == 1 and acc == 2 ** 24 + extra - 8, (xs, acc)
             scale = np.float32(xs[0]) * np.float32(ws[0])
             expect = np.float32(np.float32(sum_f32) * scale)
@@ -521,6 +521,119 @@ def pin_row_bias_once(o):
     bb = _bf16(np.array([1.5, -2.25, 0.0, 7.0, -0.125]))
     out = o.row_linear(xq, np.ones(3, np.float32), wq, np.ones(5, np.float32), bb)
     np.testing.assert_array_equal(out, np.tile(_f32(bb).astype(np.float32), (3, 1)))
+
+
+# ----------------------------------------------- modulated RMSNorm and gated residual
+
+def pin_modrms_identity_is_rmsnorm(o):
+    """scale = 0, shift = 0: the modulation is the identity (1 + 0 = 1 and n * 1 + 0 = n
+    exactly, up to the sign of a zero), so the output is the plain RMSNorm's, bit for bit
+    apart from -0 / +0, for every sample; without gamma it is the RMSNorm with gamma = 1."""
+    r = _rng(31)
+    M, K, T = 6, 256, 2
+    x = _bf16(r.standard_normal((M, K)) * np.exp(r.uniform(-4, 4, (M, 1))))
+    g = _bf16(r.uniform(0.5, 1.5, K))
+    z = np.zeros((M // T, K), np.uint16)
+    y0, r0 = o.rmsnorm(x, g, 1e-6)
+    y1, r1 = o.mod_rmsnorm(x, g, z, z, T, 1e-6)
+    np.testing.assert_array_equal(r1, r0)
+    np.testing.assert_array_equal(y1 & 0x7FFF, y0 & 0x7FFF)
+    y2, _ = o.mod_rmsnorm(x, None, z, z, T, 1e-6)
+    y3, _ = o.rmsnorm(x, _bf16(np.ones(K)), 1e-6)
+    np.testing.assert_array_equal(y2 & 0x7FFF, y3 & 0x7FFF)
+
+
+def _modrms_case(seed, M, K, T):
+    """Rows c (-1)^k with c = 2^j: with eps = 0, rstd = 2^-j exactly and n = +-1; gamma,
+    scale and shift are short dyadics, so n * gamma * (1 + scale) + shift is exact in
+    FP32 and in BF16 and the output has a closed form."""
+    r = _rng(seed)
+    js = r.integers(-6, 7, M)
+    sgn = np.where(np.arange(K) % 2 == 0, 1.0, -1.0)
+    x = (2.0 ** js)[:, None] * sgn[None, :]
+    gam = r.choice([0.5, 1.0, 2.0, 4.0], K)
+    sc = r.choice([-1.0, -0.5, 0.0, 0.25, 1.0, 3.0], (M // T, K))
+    sh = r.choice([-0.75, 0.0, 0.5, 3.0, -2.0], (M // T, K))
+    b = np.arange(M) // T
+    exact = sgn[None, :] * gam[None, :] * (1.0 + sc[b]) + sh[b]
+    return _bf16(x), _bf16(gam), _bf16(sc), _bf16(sh), exact, js
+
+
+def pin_modrms_closed_form(o):
+    """The closed form above on three samples of two rows each (so that m / T, m % 3 and
+    a transposed [K, B] modulation index all differ): every output, and rstd = 2^-j."""
+    for T, M in ((2, 6), (1, 5), (5, 5)):
+        x, g, sc, sh, exact, js = _modrms_case(40 + T, M, 96, T)
+        y, rstd = o.mod_rmsnorm(x, g, sc, sh, T, 0.0)
+        np.testing.assert_array_equal(rstd, (2.0 ** -js).astype(np.float32))
+        np.testing.assert_array_equal(_f32(y), exact)
+        # without gamma: gamma = 1 in the closed form
+        y2, _ = o.mod_rmsnorm(x, None, sc, sh, T, 0.0)
+        b = np.arange(M) // T
+        sgn = np.where(np.arange(96) % 2 == 0, 1.0, -1.0)
+        np.testing.assert_array_equal(_f32(y2), sgn[None, :] * (1.0 + _f32(sc)[b]) + _f32(sh)[b])
+
+
+def pin_modrms_error_bound(o):
+    """Random rows and modulation: within BF16 rounding (2^-9 relative) plus the FP32
+    error of the steps before it, of the float64 value x rstd gamma (1 + scale) + shift,
+    rstd itself within two FP32 ulps of the float64 formula."""
+    r = _rng(44)
+    M, K, T = 8, 384, 4
+    x = _bf16(r.standard_normal((M, K)) * np.exp(r.uniform(-3, 3, (M, 1))))
+    g = _bf16(r.uniform(0.5, 1.5, K))
+    sc = _bf16(r.standard_normal((M // T, K)) * 0.3)
+    sh = _bf16(r.standard_normal((M // T, K)) * 0.5)
+    y, rstd = o.mod_rmsnorm(x, g, sc, sh, T, 1e-6)
+    xf = _f32(x)
+    ex_r = 1.0 / np.sqrt((xf * xf).mean(1) + float(np.float32(1e-6)))
+    assert np.all(np.abs(rstd - ex_r) <= ex_r * 2.0 ** -22)
+    b = np.arange(M) // T
+    u = xf * ex_r[:, None] * _f32(g)[None, :] * (1.0 + _f32(sc)[b])
+    v = u + _f32(sh)[b]
+    err = np.abs(_f32(y) - v)
+    assert np.all(err <= np.abs(v) * 2.0 ** -8 + (np.abs(u) + np.abs(_f32(sh)[b])) * 2.0 ** -19 + 1e-38)
+    # rows of one sample use that sample's modulation row: a sub-range call agrees
+    y3, r3 = o.mod_rmsnorm(x, g, sc, sh, T, 1e-6, m0=3, rows=4)
+    np.testing.assert_array_equal(y3, y[3:7])
+    np.testing.assert_array_equal(r3, rstd[3:7])
+
+
+def pin_gated_closed_form(o):
+    """Short dyadic v, residual and gate: r + gate[m / T, n] v is exact in FP32 and BF16;
+    three samples of two rows, N = 5 (so m % 3 or a transposed gate index differ)."""
+    r = _rng(50)
+    M, N, T = 6, 5, 2
+    v = r.integers(-8, 9, (M, N)).astype(np.float32)
+    res = _bf16(r.choice([-1.5, -0.25, 0.0, 0.75, 6.0], (M, N)))
+    gate = _bf16(r.choice([-1.0, 0.0, 0.5, 2.0, 0.25], (M // T, N)))
+    out = o.gated_residual(v, res, gate, T, M)
+    b = np.arange(M) // T
+    np.testing.assert_array_equal(_f32(out), _f32(res) + _f32(gate)[b] * v)
+    # the same points given one by one, in another order
+    ms, ns = np.indices((M, N)).reshape(2, -1)
+    perm = r.permutation(ms.size)
+    o2 = o.gated_residual(v[ms[perm], ns[perm]], res[ms[perm], ns[perm]], gate, T, M,
+                          ms[perm], ns[perm])
+    np.testing.assert_array_equal(o2, out[ms[perm], ns[perm]])
+
+
+def pin_gated_special_cases(o):
+    """gate = 1, residual = 0: the output is bf16(v), the plain linear's rounding; gate =
+    0: the residual itself; and one rounding only: v = 1 + 2^-8 (a BF16 tie that rounds
+    down on its own) plus r = 2^-9 gives 1 + 2^-7, where rounding v first would give 1."""
+    r = _rng(51)
+    M, N = 4, 7
+    v = (r.standard_normal((M, N)) * 10).astype(np.float32)
+    one = _bf16(np.ones((1, N)))
+    zero = np.zeros((M, N), np.uint16)
+    np.testing.assert_array_equal(o.gated_residual(v, zero, one, M, M), o.f32_to_bf16(v))
+    res = _bf16(r.standard_normal((M, N)))
+    out = o.gated_residual(v, res, np.zeros((2, N), np.uint16), 2, M)
+    np.testing.assert_array_equal(out & 0x7FFF, res & 0x7FFF)
+    vt = np.full((1, 1), 1.0 + 2.0 ** -8, np.float32)
+    out = o.gated_residual(vt, _bf16(np.full((1, 1), 2.0 ** -9)), _bf16(np.ones((1, 1))), 1, 1)
+    assert _f32(out)[0, 0] == 1.0 + 2.0 ** -7, _f32(out)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,7 +1,7 @@
 """Plant one plausible mistake at a time in a copy of oracle.c (on the CPU), rebuild it,
 and require that some pin catches each mistake.  This shows the pins constrain every
 step of the oracle: scales, rounding, division, block indexing, per-block rescale,
-bias, RMSNorm and the BF16 fallback."""
+bias, RMSNorm, the modulated RMSNorm and gated residual, and the BF16 fallback."""
 import os
 import shutil
 
@@ -60,6 +60,24 @@ MUTANTS = [
     ("row_sum_in_double", "const float v = (float)(int32_t)acc * scale;",
      "const float v = (float)((double)acc * (double)scale);"),
     ("row_bias_twice", "return v + b;", "return v + b + b;"),
+    ("mod_scale_without_one", "const float a = 1.0f + bf16_to_f32(scale[k]);",
+     "const float a = bf16_to_f32(scale[k]);"),
+    ("mod_shift_subtracted", "yrow[k] = f32_to_bf16(u + bf16_to_f32(shift[k]));",
+     "yrow[k] = f32_to_bf16(u - bf16_to_f32(shift[k]));"),
+    ("mod_scale_shift_swapped", "gamma, scale + b * K, shift + b * K, r,",
+     "gamma, shift + b * K, scale + b * K, r,"),
+    ("mod_sample_index_modulo", "const int64_t b = m / T;", "const int64_t b = m % (M / T);"),
+    ("mod_drop_gamma", "n = n * bf16_to_f32(gamma[k]);", "n = n * 1.0f;"),
+    ("mod_shift_rounded_in", "const float u = n * a;",
+     "const float u = bf16_to_f32(f32_to_bf16(n * a));"),
+    ("gated_drop_gate", "const float gv = bf16_to_f32(gate[b * N + ns[t]]) * v[t];",
+     "const float gv = v[t];"),
+    ("gated_gate_transposed", "const float gv = bf16_to_f32(gate[b * N + ns[t]]) * v[t];",
+     "const float gv = bf16_to_f32(gate[ns[t] * (M / T) + b]) * v[t];"),
+    ("gated_sample_index_modulo", "const int64_t b = ms[t] / T;",
+     "const int64_t b = ms[t] % (M / T);"),
+    ("gated_v_rounded_first", "const float gv = bf16_to_f32(gate[b * N + ns[t]]) * v[t];",
+     "const float gv = bf16_to_f32(gate[b * N + ns[t]]) * bf16_to_f32(f32_to_bf16(v[t]));"),
 ]
 # commuted_product_noop rewrites without changing the arithmetic (FP32 multiplication
 # commutes): it checks that the harness does not report every rewrite as caught.
