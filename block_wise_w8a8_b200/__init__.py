@@ -41,6 +41,10 @@ _SIGS = {
     "w8a8_rmsnorm_quantize_act": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                   ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_rmsnorm_mod_quantize_act": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p],
     "w8a8_linear": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                     ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
@@ -171,10 +175,11 @@ def rowwise_linear(x, wq, ws, bias=None, out=None):
 
 
 def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):
-    """RMSNorm (FP64 row sums, FP32 rstd, bf16((x * rstd) * gamma)) fused with the block
-    quantizer -> (xq, xs, rstd)."""
+    """RMSNorm (FP64 row sums, FP32 rstd, bf16((x * rstd) * gamma); gamma may be None)
+    fused with the block quantizer -> (xq, xs, rstd)."""
     _need(x, torch.bfloat16, "x")
-    _need(gamma, torch.bfloat16, "gamma")
+    if gamma is not None:
+        _need(gamma, torch.bfloat16, "gamma")
     M, K = x.shape
     dev = x.device
     xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
@@ -183,6 +188,30 @@ def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):
     _check("w8a8_rmsnorm_quantize_act",
            lib().w8a8_rmsnorm_quantize_act(_ptr(x), _ptr(gamma), float(eps), M, K, _ptr(xq),
                                            _ptr(xs), _ptr(rstd), _stream(dev)))
+    return xq, xs, rstd
+
+
+def rmsnorm_mod_quantize_act(x, gamma, scale, shift, eps=1e-6, xq=None, xs=None, rstd=None):
+    """Modulated RMSNorm fused with the block quantizer: y = bf16(n * (1 + scale[b]) +
+    shift[b]) with n = x * rstd (* gamma), b = m // T, T = M // scale.shape[0] rows per
+    modulation row (a multiple of 128) -> (xq, xs, rstd)."""
+    _need(x, torch.bfloat16, "x")
+    if gamma is not None:
+        _need(gamma, torch.bfloat16, "gamma")
+    _need(scale, torch.bfloat16, "scale")
+    _need(shift, torch.bfloat16, "shift")
+    M, K = x.shape
+    B = scale.shape[0]
+    if scale.shape != (B, K) or shift.shape != (B, K) or B == 0 or M % B:
+        raise ValueError(f"scale and shift must be [B, {K}] with B dividing M = {M}")
+    dev = x.device
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
+    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=dev) if xs is None else xs
+    rstd = torch.empty((M,), dtype=torch.float32, device=dev) if rstd is None else rstd
+    _check("w8a8_rmsnorm_mod_quantize_act",
+           lib().w8a8_rmsnorm_mod_quantize_act(_ptr(x), _ptr(gamma), _ptr(scale), _ptr(shift),
+                                               M // B, float(eps), M, K, _ptr(xq), _ptr(xs),
+                                               _ptr(rstd), _stream(dev)))
     return xq, xs, rstd
 
 

@@ -6,7 +6,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "w8a8.cu")
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("w8a8.cu", "common.cuh", "gemm.cuh", "quant.cuh")] + \
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("w8a8.cu", "common.cuh", "gemm.cuh", "norm.cuh", "quant.cuh")] + \
     [os.path.join(ROOT, "include", "w8a8.h")]
 LIB = os.path.join(HERE, "libw8a8.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -10,6 +10,7 @@
 #include "../../include/w8a8.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "norm.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -27,6 +28,8 @@ struct DeviceInfo {
     int sms = 0;
     bool gemm_attr_set[4] = {false, false, false, false};
     bool quant_attr_set = false;
+    bool norm_attr_set[4] = {false, false, false, false};
+    int norm_max_clusters[norm::kMaxCluster + 1] = {};    // by cluster size, 0 = unknown
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -326,6 +329,92 @@ w8a8_status_t noalloc_scratch(int dev, void *&ptr)
     return W8A8_OK;
 }
 
+// Fused RMSNorm (+ modulation) + block quantization: clusters of C = min(8, K / 128) CTAs,
+// one cluster per 128-row strip at a time, as many clusters as fit on the device.
+template <bool kMod, bool kExactSq>
+w8a8_status_t launch_norm(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
+{
+    int dev;
+    W8A8_TRY(current_device(dev));
+    CUtensorMap tm;
+    W8A8_TRY(make_map(tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.MB * 128, p.K, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+    auto kern = norm::rmsnorm_quantize_kernel<kMod, kExactSq>;
+    const int C = static_cast<int>(std::min<int64_t>(norm::kMaxCluster, p.K / 128));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(C);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.blockDim = dim3(norm::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = norm::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int max_clusters;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const int v = static_cast<int>(kMod) * 2 + static_cast<int>(kExactSq);
+        if (!g_dev[dev].norm_attr_set[v]) {
+            const cudaError_t e = cudaFuncSetAttribute(
+                kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(norm::kSmemBytes));
+            if (e != cudaSuccess)
+                return cuda_fail(e);
+            g_dev[dev].norm_attr_set[v] = true;
+        }
+        if (g_dev[dev].norm_max_clusters[C] == 0) {
+            int n = 0;
+            cfg.gridDim = dim3(static_cast<unsigned>(C * g_dev[dev].sms), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+                cudaGetLastError();
+                n = g_dev[dev].sms / C;
+            }
+            g_dev[dev].norm_max_clusters[C] = std::max(1, n);
+        }
+        max_clusters = g_dev[dev].norm_max_clusters[C];
+    }
+    const int64_t nclusters = std::max<int64_t>(1, std::min<int64_t>(p.MB, max_clusters));
+    cfg.gridDim = dim3(static_cast<unsigned>(nclusters * C), 1, 1);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tm, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    return launch_status();
+}
+
+// Checks shared by both RMSNorm entry points; fills p (except the modulation fields).
+w8a8_status_t norm_common(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma, float eps, int64_t M,
+                          int64_t K, int8_t *xq, float *xs, float *rstd_out, norm::Params &p)
+{
+    if (M < 0 || K < 0 || !(eps >= 0.0f) || !(eps <= 3.4e38f))
+        return W8A8_ERR_INVALID_ARG;
+    if (M % 128 || K % 128 || M > kMaxTmaCoord || K > kMaxTmaCoord)
+        return W8A8_ERR_SHAPE;
+    if (M > 0 && K == 0)
+        return W8A8_ERR_SHAPE;
+    if (M == 0)
+        return W8A8_OK;
+    W8A8_TRY(check_device_ptr(x));
+    if (gamma != nullptr)
+        W8A8_TRY(check_device_ptr(gamma));
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(xs));
+    if (rstd_out != nullptr)
+        W8A8_TRY(check_device_ptr(rstd_out));
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(xq) ||
+        (reinterpret_cast<uintptr_t>(xs) & 3u) || (reinterpret_cast<uintptr_t>(rstd_out) & 3u))
+        return W8A8_ERR_ALIGNMENT;
+    p = norm::Params{};
+    p.gamma = gamma;
+    p.eps = eps;
+    p.MB = M / 128;
+    p.K = K;
+    p.q = xq;
+    p.s = xs;
+    p.rstd_out = rstd_out;
+    return W8A8_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -348,50 +437,36 @@ w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t 
                                         float eps, int64_t M, int64_t K, int8_t *xq, float *xs,
                                         float *rstd_out, void *stream)
 {
-    if (M < 0 || K < 0 || !(eps >= 0.0f))
+    norm::Params p;
+    W8A8_TRY(norm_common(x, gamma, eps, M, K, xq, xs, rstd_out, p));
+    if (M == 0)
+        return W8A8_OK;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return eps == 0.0f ? launch_norm<false, true>(x, p, st) : launch_norm<false, false>(x, p, st);
+}
+
+w8a8_status_t w8a8_rmsnorm_mod_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
+                                            const w8a8_bf16_t *scale, const w8a8_bf16_t *shift,
+                                            int64_t T, float eps, int64_t M, int64_t K,
+                                            int8_t *xq, float *xs, float *rstd_out, void *stream)
+{
+    if (T <= 0)
         return W8A8_ERR_INVALID_ARG;
-    if (M % 128 || K % 128 || K > 16384)
+    norm::Params p;
+    W8A8_TRY(norm_common(x, gamma, eps, M, K, xq, xs, rstd_out, p));
+    if (T % 128 || M % T)
         return W8A8_ERR_SHAPE;
     if (M == 0)
         return W8A8_OK;
-    if (K == 0)
-        return W8A8_ERR_SHAPE;
-    W8A8_TRY(check_device_ptr(x));
-    W8A8_TRY(check_device_ptr(gamma));
-    W8A8_TRY(check_device_ptr(xq));
-    W8A8_TRY(check_device_ptr(xs));
-    if (rstd_out != nullptr)
-        W8A8_TRY(check_device_ptr(rstd_out));
-    if (!aligned16(x) || !aligned16(gamma) || !aligned16(xq) ||
-        (reinterpret_cast<uintptr_t>(xs) & 3u) || (reinterpret_cast<uintptr_t>(rstd_out) & 3u))
+    W8A8_TRY(check_device_ptr(scale));
+    W8A8_TRY(check_device_ptr(shift));
+    if (!aligned16(scale) || !aligned16(shift))
         return W8A8_ERR_ALIGNMENT;
-    int dev;
-    W8A8_TRY(current_device(dev));
-    const int64_t MB = M / 128;
-    int max_clusters = 0;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(quant::kNormCluster * 64, 1, 1);
-        cfg.blockDim = dim3(quant::kThreads, 1, 1);
-        cudaLaunchAttribute attr;
-        attr.id = cudaLaunchAttributeClusterDimension;
-        attr.val.clusterDim.x = quant::kNormCluster;
-        attr.val.clusterDim.y = 1;
-        attr.val.clusterDim.z = 1;
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, quant::rmsnorm_quantize_kernel, &cfg) !=
-                cudaSuccess ||
-            max_clusters <= 0) {
-            cudaGetLastError();
-            max_clusters = g_dev[dev].sms / quant::kNormCluster;
-        }
-    }
-    const int64_t nclusters = std::max<int64_t>(1, std::min<int64_t>(MB, max_clusters));
-    quant::rmsnorm_quantize_kernel<<<static_cast<unsigned>(nclusters * quant::kNormCluster),
-                                     quant::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        x, gamma, eps, MB, K, xq, xs, rstd_out);
-    return launch_status();
+    p.scale = scale;
+    p.shift = shift;
+    p.T = T;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return eps == 0.0f ? launch_norm<true, true>(x, p, st) : launch_norm<true, false>(x, p, st);
 }
 
 size_t w8a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N)

@@ -111,11 +111,31 @@ W8A8_API w8a8_status_t w8a8_quantize_act(const w8a8_bf16_t *x, int64_t M, int64_
  *     rstd[m] = fp32( 1 / sqrt( (sum_k x[m,k]^2) / K + eps ) )   (sum and sqrt in FP64)
  *     y[m,k]  = bf16( (x[m,k] * rstd[m]) * gamma[k] )            (FP32 products)
  *   and y is block-quantized exactly as by w8a8_quantize_act, without being stored.
- *   x [M, K] BF16, gamma [K] BF16 -> xq [M, K] INT8, xs [M/128, K/128] FP32, and
- *   rstd_out [M] FP32 when not NULL.  M, K multiples of 128; K <= 16384. */
+ *   x [M, K] BF16, gamma [K] BF16 or NULL (then y = bf16(x * rstd)) -> xq [M, K] INT8,
+ *   xs [M/128, K/128] FP32, and rstd_out [M] FP32 when not NULL.
+ *   M, K multiples of 128 (else W8A8_ERR_SHAPE; M == 0 is a no-op), eps >= 0 and finite
+ *   (else W8A8_ERR_INVALID_ARG); x, gamma, xq 16-byte aligned, xs and rstd_out 4-byte
+ *   aligned.  Reads x once from HBM when K <= 6144 (the strip's blocks stay on chip
+ *   between the two passes), twice (the second from L2) above that. */
 W8A8_API w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
                                         float eps, int64_t M, int64_t K, int8_t *xq,
                                         float *xs, float *rstd_out, void *stream);
+
+/* Modulated RMSNorm (adaptive scale-shift of diffusion transformers) fused ahead of the
+ * activation quantizer (TurboT2VA paper, fused-operator paragraph: modulated RMS
+ * normalization and scale-shift modulation, with modality- and timestep-dependent
+ * modulation; the page gives no formula, this is the adaptive-norm form).  Rows come in
+ * groups of T consecutive rows (one sample's tokens) sharing one modulation row b = m / T:
+ *     n[m,k]  = fl(x[m,k] * rstd[m]), times gamma[k] (FP32 product) when gamma != NULL
+ *     y[m,k]  = bf16( fl( fl(n[m,k] * fl(1 + scale[b,k])) + shift[b,k] ) )
+ *   with rstd as above, and y block-quantized as by w8a8_quantize_act, not stored.
+ *   scale, shift [M/T, K] BF16 device buffers, 16-byte aligned.  T > 0 (else
+ *   W8A8_ERR_INVALID_ARG), T a multiple of 128 dividing M (else W8A8_ERR_SHAPE); the
+ *   other arguments as for w8a8_rmsnorm_quantize_act. */
+W8A8_API w8a8_status_t w8a8_rmsnorm_mod_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
+                                            const w8a8_bf16_t *scale, const w8a8_bf16_t *shift,
+                                            int64_t T, float eps, int64_t M, int64_t K,
+                                            int8_t *xq, float *xs, float *rstd_out, void *stream);
 
 /* Bytes of device workspace w8a8_linear needs for an M x K activation on the INT8 path:
  * the INT8 codes (M*K bytes, rounded up to 256) followed by the FP32 scales.  Returns 0

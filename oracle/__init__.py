@@ -56,7 +56,7 @@ def load(path=None):
                  "oracle_w8a8_linear_at", "oracle_rmsnorm", "oracle_rmsnorm_apply",
                  "oracle_bf16_linear", "oracle_bf16_linear_at", "oracle_num_threads",
                  "oracle_row_quantize", "oracle_row_linear", "oracle_row_linear_at",
-                 "oracle_mod_rmsnorm", "oracle_gated_residual"]:
+                 "oracle_mod_rmsnorm", "oracle_mod_rmsnorm_apply", "oracle_gated_residual"]:
         getattr(lib, name).restype = ctypes.c_int
     lib.oracle_f32_to_bf16.restype = None
     if path is None:
@@ -205,6 +205,24 @@ class Oracle:
         if rc:
             raise ValueError("mod_rmsnorm: bad arguments")
         return y, rstd
+
+    def mod_rmsnorm_apply(self, x_bits, gamma_bits, scale_bits, shift_bits, T, rstd, m0=0):
+        """mod_rmsnorm's normalisation with a given rstd for rows m0 .. m0 + rstd.size."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        g = None if gamma_bits is None else np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+        sc = np.ascontiguousarray(scale_bits, dtype=np.uint16)
+        sh = np.ascontiguousarray(shift_bits, dtype=np.uint16)
+        r = np.ascontiguousarray(rstd, dtype=np.float32)
+        M, K = x.shape
+        if T <= 0 or M % T or sc.shape != (M // T, K) or sh.shape != (M // T, K):
+            raise ValueError("mod_rmsnorm_apply: bad shapes")
+        y = np.empty((r.size, K), dtype=np.uint16)
+        rc = self.lib.oracle_mod_rmsnorm_apply(_ptr(x), _ptr(g), _ptr(sc), _ptr(sh), _i64(T),
+                                               _ptr(r), _i64(M), _i64(K), _i64(m0),
+                                               _i64(r.size), _ptr(y))
+        if rc:
+            raise ValueError("mod_rmsnorm_apply: bad arguments")
+        return y
 
     def gated_residual(self, v, r_bits, gate_bits, T, M, ms=None, ns=None):
         """out = bf16(fl(r + fl(gate[m / T, n] * v))).  With ms, ns: v and r_bits hold the

@@ -26,6 +26,8 @@
  *     inference-stack section, guard paragraph.
  *   - The per-row / per-output-channel post-scale operator (the paper's own W8A8
  *     kernel): TurboT2VA paper, W8A8 operator paragraph (see the per-row section).
+ *   - Modulated RMSNorm (adaptive scale-shift) and the gated residual update: TurboT2VA
+ *     paper, fused-operator paragraph (see the modulated-RMSNorm section).
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   rounding of x/s to an integer is round-half-to-even; x/s is one IEEE FP32 division
@@ -34,7 +36,9 @@
  *   by that product, and the K blocks are summed in ascending order in FP32 with no
  *   fused multiply-add; the bias (BF16 widened to FP32) is added once at the end.
  *   RMSNorm: sum of squares in FP64, rstd = 1/sqrt(mean + eps) in FP64 rounded to FP32,
- *   normalised value = bf16((x * rstd) * gamma) with FP32 products.
+ *   normalised value = bf16((x * rstd) * gamma) with FP32 products.  Modulated RMSNorm:
+ *   bf16(fl(fl(n * fl(1 + scale)) + shift)) with one modulation row per T-row sample;
+ *   gated residual: bf16(fl(r + fl(gate * v))) on the unrounded FP32 linear output v.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -fPIC -shared.
  * OpenMP splits only independent outputs, so the thread count never changes a bit.
@@ -360,6 +364,22 @@ int oracle_mod_rmsnorm(const uint16_t *x, const uint16_t *gamma, const uint16_t 
         const float r = row_rstd(x + m * K, K, eps);
         rstd[i] = r;
         row_apply_mod(x + m * K, gamma, scale + b * K, shift + b * K, r, K, y + i * K);
+    }
+    return 0;
+}
+
+/* Same modulated normalisation with a given per-row rstd (rows [m0, m0 + rows), rstd[i]). */
+int oracle_mod_rmsnorm_apply(const uint16_t *x, const uint16_t *gamma, const uint16_t *scale,
+                             const uint16_t *shift, int64_t T, const float *rstd, int64_t M,
+                             int64_t K, int64_t m0, int64_t rows, uint16_t *y)
+{
+    if (K <= 0 || T <= 0 || M % T != 0 || m0 < 0 || rows < 0 || m0 + rows > M)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < rows; ++i) {
+        const int64_t m = m0 + i;
+        const int64_t b = m / T;
+        row_apply_mod(x + m * K, gamma, scale + b * K, shift + b * K, rstd[i], K, y + i * K);
     }
     return 0;
 }

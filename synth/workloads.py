@@ -13,6 +13,7 @@ from .philox import philox4x32_10, uniform_open01, normal_pairs
 
 # Stream ids (the second key word).
 STREAM_X, STREAM_W, STREAM_BIAS, STREAM_GAMMA, STREAM_OUTLIER = 0, 1, 2, 3, 4
+STREAM_MOD_SCALE, STREAM_MOD_SHIFT, STREAM_GATE, STREAM_RESID = 5, 6, 7, 8
 STREAM_LAYER0 = 16          # chained linears use 16, 17, ...
 STREAM_X_K2000, STREAM_W_K2000 = 32, 33
 
@@ -142,6 +143,19 @@ class _Workload:
 
     def gamma(self, K):
         return uniform_bf16(1, K, self.seed, STREAM_GAMMA, 0.5, 1.5).reshape(-1)
+
+    def modulation(self, B, K, sigma=0.5):
+        """Per-sample scale and shift rows [B, K] of the adaptive norm, N(0, sigma) each."""
+        return (normal_bf16(B, K, self.seed, STREAM_MOD_SCALE, sigma),
+                normal_bf16(B, K, self.seed, STREAM_MOD_SHIFT, sigma))
+
+    def gate(self, B, N, sigma=0.5):
+        """Per-sample gate rows [B, N] of the gated residual update, N(0, sigma)."""
+        return normal_bf16(B, N, self.seed, STREAM_GATE, sigma)
+
+    def residual(self, M, N, row0=0, nrows=None):
+        """The residual stream [M, N] that a gated update adds to, N(0, 1)."""
+        return normal_bf16(M, N, self.seed, STREAM_RESID, 1.0, row0, nrows)
 
 
 def _lin(name, M, K, N, w_stream, w_sigma, bias=None):

@@ -593,10 +593,12 @@ def pin_modrms_error_bound(o):
     v = u + _f32(sh)[b]
     err = np.abs(_f32(y) - v)
     assert np.all(err <= np.abs(v) * 2.0 ** -8 + (np.abs(u) + np.abs(_f32(sh)[b])) * 2.0 ** -19 + 1e-38)
-    # rows of one sample use that sample's modulation row: a sub-range call agrees
+    # rows of one sample use that sample's modulation row: a sub-range call agrees, and
+    # so does the normalisation applied with the returned rstd
     y3, r3 = o.mod_rmsnorm(x, g, sc, sh, T, 1e-6, m0=3, rows=4)
     np.testing.assert_array_equal(y3, y[3:7])
     np.testing.assert_array_equal(r3, rstd[3:7])
+    np.testing.assert_array_equal(o.mod_rmsnorm_apply(x, g, sc, sh, T, rstd[3:7], m0=3), y[3:7])
 
 
 def pin_gated_closed_form(o):

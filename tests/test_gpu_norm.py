@@ -1,0 +1,158 @@
+"""The fused RMSNorm + block quantizer, plain and modulated (TurboDiffusion article,
+inference list item 5; TurboT2VA paper, fused-operator paragraph), on the GPU through the
+C ABI, against the oracle.
+
+rstd must equal the oracle's bit for bit except on rows where the two FP64 sums, taken in
+different orders, round to neighbouring FP32 values (at most one ulp, on a vanishing
+fraction of rows); given the kernel's rstd, codes and scales must equal the oracle's bit
+for bit.  Shapes cover every cluster size (C = min(8, K / 128)), blocks resident between
+the passes (K / 128 / C <= 6) and reloaded, block counts per CTA that are not a multiple
+of the four consumer groups, CTAs with no block, gamma absent, and eps = 0 (the exact
+conversion path)."""
+import numpy as np
+import pytest
+import torch
+
+import block_wise_w8a8_b200 as w8
+from gpu_util import dev_bf16
+from synth import f64_to_bf16_bits, workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _no_device_error():
+    yield
+    assert w8.device_error() == 0
+
+
+def _rows(shape, seed, zero_row=True, tiny_row=True):
+    r = np.random.default_rng(seed)
+    x = r.standard_normal(shape) * np.exp(r.uniform(-4, 4, (shape[0], 1)))
+    if zero_row:
+        x[0] = 0.0                                  # rstd = 1 / sqrt(eps)
+    if tiny_row and shape[0] > 1:
+        x[1] = r.standard_normal(shape[1]) * 1e-39  # subnormal BF16 values
+    if shape[0] > 2:
+        x[2, ::3] = 0.0                             # zeros inside a row
+    return f64_to_bf16_bits(x)
+
+
+def _check(orc, x, g, eps, xq, xs, rstd, mod=None):
+    """mod = (scale_bits, shift_bits, T) for the modulated operation."""
+    if mod is None:
+        _, r_ref = orc.rmsnorm(x, g if g is not None else f64_to_bf16_bits(np.ones(x.shape[1])), eps)
+    else:
+        _, r_ref = orc.mod_rmsnorm(x, g, mod[0], mod[1], mod[2], eps)
+    diff = np.nonzero(rstd.view(np.uint32) != r_ref.view(np.uint32))[0]
+    assert diff.size <= max(1, rstd.size // 100000), diff[:10]
+    for i in diff:
+        assert abs(int(rstd.view(np.int32)[i]) - int(r_ref.view(np.int32)[i])) <= 1
+    if mod is None:
+        gg = g if g is not None else f64_to_bf16_bits(np.ones(x.shape[1]))
+        y = orc.rmsnorm_apply(x, gg, rstd)
+    else:
+        y = orc.mod_rmsnorm_apply(x, g, mod[0], mod[1], mod[2], rstd)
+    q_ref, s_ref = orc.block_quantize(y)
+    np.testing.assert_array_equal(xs.view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(xq, q_ref)
+
+
+SHAPES = [(128, 128),      # C = 1
+          (256, 384),      # C = 3
+          (384, 896),      # C = 7, one block per CTA
+          (256, 6144),     # C = 8, six blocks per CTA: resident, the largest
+          (256, 7168),     # seven blocks per CTA: reloaded, not a multiple of 4
+          (128, 8192),     # eight blocks per CTA: reloaded
+          (1152, 2048)]    # more strips than one pass of clusters on small M
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+@pytest.mark.parametrize("with_gamma", [True, False])
+def test_rmsnorm_quantize(orc, M, K, with_gamma):
+    x = _rows((M, K), M * 7 + K)
+    g = f64_to_bf16_bits(np.random.default_rng(K).uniform(0.5, 1.5, K)) if with_gamma else None
+    xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), None if g is None else dev_bf16(g), 1e-6)
+    _check(orc, x, g, 1e-6, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy())
+
+
+@pytest.mark.parametrize("M,K,T", [(256, 384, 128), (384, 896, 384), (512, 6144, 256),
+                                   (256, 7168, 128), (640, 1024, 128)])
+@pytest.mark.parametrize("with_gamma", [True, False])
+def test_mod_rmsnorm_quantize(orc, M, K, T, with_gamma):
+    r = np.random.default_rng(M + K + T)
+    x = _rows((M, K), M * 5 + K)
+    g = f64_to_bf16_bits(r.uniform(0.5, 1.5, K)) if with_gamma else None
+    sc = f64_to_bf16_bits(r.standard_normal((M // T, K)) * 0.5)
+    sh = f64_to_bf16_bits(r.standard_normal((M // T, K)) * 0.5)
+    sc[0, :7] = f64_to_bf16_bits(np.full(7, -1.0))   # 1 + scale = 0: y = shift
+    xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), None if g is None else dev_bf16(g),
+                                               dev_bf16(sc), dev_bf16(sh), 1e-6)
+    _check(orc, x, g, 1e-6, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(), (sc, sh, T))
+
+
+@pytest.mark.parametrize("modulated", [False, True])
+def test_eps_zero_exact_squares(orc, modulated):
+    """eps = 0 takes the exact FP64 conversion: rows of subnormal and mixed magnitudes."""
+    M, K = 256, 1024
+    x = _rows((M, K), 99, zero_row=False)
+    # row 1 is subnormal but for one normal value, so that rstd stays finite
+    x[1, 5] = f64_to_bf16_bits(np.array([1.0]))[0]
+    x[3, 0] = f64_to_bf16_bits(np.array([2.0 ** -126]))[0]
+    g = f64_to_bf16_bits(np.random.default_rng(5).uniform(0.5, 1.5, K))
+    if modulated:
+        r = np.random.default_rng(6)
+        sc = f64_to_bf16_bits(r.standard_normal((2, K)) * 0.5)
+        sh = f64_to_bf16_bits(r.standard_normal((2, K)) * 0.5)
+        xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), dev_bf16(g), dev_bf16(sc),
+                                                   dev_bf16(sh), 0.0)
+        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(), (sc, sh, 128))
+    else:
+        xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), dev_bf16(g), 0.0)
+        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy())
+
+
+@pytest.mark.parametrize("modulated", [False, True])
+def test_hires_chain_norm_sampled(orc, modulated):
+    """The M = 32768, K = 4096 chain input (one sample, T = M): the whole launch runs, and
+    three 128-row strips (first, one in the middle, last) match the oracle."""
+    wl = workload("hires_chain_32768")
+    M, K = 32768, 4096
+    eps = wl.extra["eps"]
+    x = wl.x(M, K)
+    g = wl.gamma(K)
+    if modulated:
+        sc, sh = wl.modulation(1, K)
+        xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), dev_bf16(g), dev_bf16(sc),
+                                                   dev_bf16(sh), eps)
+    else:
+        xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), dev_bf16(g), eps)
+    xq, xs, rstd = xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy()
+    for mb in (0, 137, 255):
+        rows = slice(mb * 128, (mb + 1) * 128)
+        xr = x[rows]
+        if modulated:
+            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows], (sc, sh, 128))
+        else:
+            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows])
+
+
+def test_mod_errors():
+    L = w8.lib()
+    st = w8._stream(torch.device("cuda"))
+    x = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
+    m = torch.zeros((2, 256), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((256, 256), dtype=torch.int8, device="cuda")
+    s = torch.empty((2, 2), dtype=torch.float32, device="cuda")
+    f = L.w8a8_rmsnorm_mod_quantize_act
+    P = lambda t: t.data_ptr()
+    assert f(P(x), None, P(m), P(m), 128, 1e-6, 256, 256, P(q), P(s), None, st) == 0
+    assert f(P(x), None, P(m), P(m), 0, 1e-6, 256, 256, P(q), P(s), None, st) == 1
+    assert f(P(x), None, P(m), P(m), 64, 1e-6, 256, 256, P(q), P(s), None, st) == 2
+    assert f(P(x), None, P(m), P(m), 384, 1e-6, 256, 256, P(q), P(s), None, st) == 2
+    assert f(P(x), None, P(m) + 2, P(m), 128, 1e-6, 256, 256, P(q), P(s), None, st) == 4
+    host = torch.zeros((2, 256), dtype=torch.bfloat16)
+    assert f(P(x), None, P(m), P(host), 128, 1e-6, 256, 256, P(q), P(s), None, st) == 3
+    assert f(P(x), None, P(m), P(m), 128, -1.0, 256, 256, P(q), P(s), None, st) == 1
+    assert L.w8a8_rmsnorm_quantize_act(P(x), None, 1e-6, 256, 200, P(q), P(s), None, st) == 2
+    torch.cuda.synchronize()

@@ -66,7 +66,8 @@ MUTANTS = [
      "yrow[k] = f32_to_bf16(u - bf16_to_f32(shift[k]));"),
     ("mod_scale_shift_swapped", "gamma, scale + b * K, shift + b * K, r,",
      "gamma, shift + b * K, scale + b * K, r,"),
-    ("mod_sample_index_modulo", "const int64_t b = m / T;", "const int64_t b = m % (M / T);"),
+    ("mod_sample_index_modulo", "const int64_t b = m / T;\n        const float r = row_rstd(",
+     "const int64_t b = m % (M / T);\n        const float r = row_rstd("),
     ("mod_drop_gamma", "n = n * bf16_to_f32(gamma[k]);", "n = n * 1.0f;"),
     ("mod_shift_rounded_in", "const float u = n * a;",
      "const float u = bf16_to_f32(f32_to_bf16(n * a));"),
