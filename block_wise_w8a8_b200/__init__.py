@@ -45,6 +45,10 @@ _SIGS = {
                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p],
+    "w8a8_linear_prequant_gated": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                   ctypes.c_int64, ctypes.POINTER(_Weight), ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                   ctypes.c_void_p, ctypes.c_void_p],
     "w8a8_linear": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                     ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
@@ -288,6 +292,25 @@ def linear_prequant(xq, xs, weight, bias=None, out=None):
     out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=xq.device) if out is None else out
     _check("w8a8_linear_prequant", lib().w8a8_linear_prequant(
         _ptr(xq), _ptr(xs), M, K, weight.record(), _ptr(bias), _ptr(out), _stream(xq.device)))
+    return out
+
+
+def linear_prequant_gated(xq, xs, weight, resid, gate, bias=None, out=None):
+    """The INT8 block-scaled GEMM with the gated residual update in its epilogue:
+    out = bf16(resid + gate[m // T] * (xq wq^T + bias)), T = M // gate.shape[0].  out may
+    be resid itself (in-place update); by default a new tensor."""
+    _need(xq, torch.int8, "xq")
+    _need(xs, torch.float32, "xs")
+    _need(resid, torch.bfloat16, "resid")
+    _need(gate, torch.bfloat16, "gate")
+    M, K = xq.shape
+    B = gate.shape[0]
+    if resid.shape != (M, weight.N) or gate.shape != (B, weight.N) or B == 0 or M % B:
+        raise ValueError(f"resid must be [{M}, {weight.N}] and gate [B, {weight.N}] with B dividing M")
+    out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _check("w8a8_linear_prequant_gated", lib().w8a8_linear_prequant_gated(
+        _ptr(xq), _ptr(xs), M, K, weight.record(), _ptr(bias), _ptr(resid), _ptr(gate), M // B,
+        _ptr(out), _stream(xq.device)))
     return out
 
 

@@ -8,6 +8,8 @@
 //               product P[m,n,kb] of the INT8 codes is formed by tcgen05.mma kind::i8 in
 //               tensor memory, then the epilogue warps add float(P) * (xs * ws) into FP32
 //               running sums held in registers.  After the last block: + bias, BF16 store.
+//   kI8Gated  : kI8Scaled with the gated residual update of the TurboT2VA paper's fused-
+//               operator paragraph in the epilogue: y = bf16(r + gate[m / T] * v).
 //   kI8Dump   : same main loop; the epilogue writes P[m,n,kb] itself (test hook).
 //   kBf16     : BF16 x BF16 -> FP32 GEMM (kind::f16) for the guard's fallback (TurboT2VA
 //               paper, guard paragraph), FP32 accumulation over all of K in tensor memory.
@@ -41,7 +43,7 @@
 namespace w8a8 {
 namespace gemm {
 
-enum class Mode : int { kI8Scaled = 0, kI8Dump = 1, kBf16 = 2, kI8Row = 3 };
+enum class Mode : int { kI8Scaled = 0, kI8Dump = 1, kBf16 = 2, kI8Row = 3, kI8Gated = 4 };
 
 constexpr int BM = 128;
 constexpr int BN = 256;
@@ -74,10 +76,21 @@ struct alignas(1024) Smem {
     uint64_t tempty[2];
     uint64_t mma_done;
     uint64_t sready[2];            // scale table sprod[b] written (all epilogue threads)
+    alignas(16) uint8_t stage[8][32 * 64];   // per epilogue warp: 32 rows x 64 bytes
     uint32_t tmem_base;
     int abort;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+
+// Byte offset of 16-byte piece c (0..3) of row r (0..31) in an epilogue warp's staging
+// buffer: rows of 64 bytes, pieces XOR-swizzled with (r / 2) % 4, so that a warp writing
+// one piece of each of its 32 rows, or reading 4 pieces of 8 rows, hits 32 distinct banks
+// in every quarter-warp phase.
+__device__ __forceinline__ uint32_t stage_off(int r, int c)
+{
+    return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
 
 struct Params {
     int64_t M, N, K;
@@ -86,6 +99,11 @@ struct Params {
     const float *ws;          // [N/128, K/128] (INT8 modes)
     const uint16_t *bias;     // [N] BF16 or null
     uint16_t *y;              // [M, N] BF16
+    // Gated residual (kI8Gated): y = bf16(fl(resid + fl(gate[m / gate_T] * v))) with v the
+    // FP32 output of kI8Scaled; resid may be y itself.
+    const uint16_t *resid;    // [M, N] BF16
+    const uint16_t *gate;     // [M / gate_T, N] BF16
+    int64_t gate_T;
     int32_t *dump;            // [M, N, K/128] (dump mode)
 };
 
@@ -98,6 +116,27 @@ __device__ __forceinline__ void tile_coords(int t, int num_tm, int num_tn, int &
     const int local = t - group * per_group;
     tm = first + local % gsz;
     tn = local / gsz;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Eight BF16 bias values (or zeros) as FP32.
+__device__ __forceinline__ void load_bias8(const uint16_t *bias, int64_t n, float (&bb)[8])
+{
+    if (bias != nullptr) {
+        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(bias + n));
+        bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
+        bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
+        bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
+        bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            bb[i] = 0.0f;
+    }
 }
 
 // The block scales a tile needs, copied global -> shared with cp.async by the epilogue
@@ -138,7 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const Params p)
 {
     constexpr bool kInt8 = (kMode != Mode::kBf16);                    // INT8 operands
-    constexpr bool kPerKb = (kMode == Mode::kI8Scaled || kMode == Mode::kI8Dump);   // per-K-block sums
+    constexpr bool kPerKb = (kMode == Mode::kI8Scaled || kMode == Mode::kI8Dump ||
+                             kMode == Mode::kI8Gated);                // per-K-block sums
+    constexpr bool kScaled = (kMode == Mode::kI8Scaled || kMode == Mode::kI8Gated);
     constexpr int kSliceElems = kInt8 ? 128 : 64;
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -292,7 +333,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
 
         uint32_t acc_i = 0;
-        if (kMode == Mode::kI8Scaled) {
+        if (kScaled) {
             const int KB = static_cast<int>(p.K / 128);
             constexpr int kEpiThreads = NUM_EPI_WARPS * 32;
             if (static_cast<int>(blockIdx.x) < p.num_tiles) {
@@ -318,6 +359,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     int tm2, tn2;
                     tile_coords(tnext, p.num_tm, p.num_tn, tm2, tn2);
                     scales_fetch(sm.sx[sb ^ 1], sm.sw[sb ^ 1], p, tm2, tn2, etid, kEpiThreads);
+                }
+                if (kMode == Mode::kI8Gated) {
+                    const int64_t pm = static_cast<int64_t>(tm) * BM + row;
+                    const int64_t pn = static_cast<int64_t>(tn) * BN + half * 128;
+                    if (pn < p.N) {
+                        prefetch_l2(p.resid + pm * p.N + pn);
+                        prefetch_l2(p.resid + pm * p.N + pn + 64);
+                    }
                 }
                 float2 acc[64];
 #pragma unroll
@@ -359,31 +408,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 cp_async_wait_all();
                 mbar_arrive(&sm.sready[sb ^ 1]);
-                // bias + BF16 store: this thread owns row m, columns n0 .. n0 + 127
+                // bias (+ gated residual) + BF16 store.  This thread owns row m, columns
+                // n0 .. n0 + 127; its warp owns rows m_w .. m_w + 31 of those columns.  The
+                // warp writes them in four rounds of 32 columns through its staging buffer:
+                // each thread puts its row's 64 bytes there, then the warp stores 64-byte
+                // row segments, 8 rows per instruction (8 cache lines instead of 32).  The
+                // gated mode reads the residual the same way in reverse.
                 const int64_t m = static_cast<int64_t>(tm) * BM + row;
                 const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                const int64_t m_w = m - static_cast<int64_t>(lane);
                 if (n0 < p.N) {
-                    uint16_t *dst = p.y + m * p.N + n0;
+                    uint8_t *stg = sm.stage[ew];
+                    const int pr = static_cast<int>(lane >> 2), pc = static_cast<int>(lane & 3);
+                    const uint16_t *gp = kMode == Mode::kI8Gated ? p.gate + (m / p.gate_T) * p.N + n0 : nullptr;
 #pragma unroll
-                    for (int c8 = 0; c8 < 16; ++c8) {
-                        float bb[8];
-                        if (p.bias != nullptr) {
-                            const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + n0 + c8 * 8));
-                            bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
-                            bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
-                            bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
-                            bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
-                        } else {
+                    for (int rd = 0; rd < 4; ++rd) {
+                        const int64_t ncol = n0 + rd * 32;
+                        if (kMode == Mode::kI8Gated) {
+                            // the residual's 32 x 32 block, 64-byte row segments
+                            uint4 rv[4];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                bb[i] = 0.0f;
+                            for (int j = 0; j < 4; ++j)
+                                rv[j] = *reinterpret_cast<const uint4 *>(p.resid + (m_w + 8 * j + pr) * p.N + ncol + pc * 8);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                st_shared_v4(stg + stage_off(8 * j + pr, pc), rv[j]);
+                            __syncwarp();
                         }
-                        uint4 o;
-                        o.x = pack_bf16x2(acc[c8 * 4 + 0].x + bb[0], acc[c8 * 4 + 0].y + bb[1]);
-                        o.y = pack_bf16x2(acc[c8 * 4 + 1].x + bb[2], acc[c8 * 4 + 1].y + bb[3]);
-                        o.z = pack_bf16x2(acc[c8 * 4 + 2].x + bb[4], acc[c8 * 4 + 2].y + bb[5]);
-                        o.w = pack_bf16x2(acc[c8 * 4 + 3].x + bb[6], acc[c8 * 4 + 3].y + bb[7]);
-                        *reinterpret_cast<uint4 *>(dst + c8 * 8) = o;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int c8 = rd * 4 + c;
+                            float bb[8];
+                            load_bias8(p.bias, n0 + c8 * 8, bb);
+                            uint32_t o[4];
+                            if (kMode == Mode::kI8Gated) {
+                                // gated residual update (TurboT2VA paper, fused-operator
+                                // paragraph): one rounding for the product, one for the sum
+                                const uint4 gv = __ldg(reinterpret_cast<const uint4 *>(gp + c8 * 8));
+                                const uint4 rv = ld_shared_v4(stg + stage_off(static_cast<int>(lane), c));
+                                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                                const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float v0 = acc[c8 * 4 + i].x + bb[2 * i];
+                                    const float v1 = acc[c8 * 4 + i].y + bb[2 * i + 1];
+                                    o[i] = pack_bf16x2(__fadd_rn(bf16_lo(rw[i]), __fmul_rn(bf16_lo(gw[i]), v0)),
+                                                       __fadd_rn(bf16_hi(rw[i]), __fmul_rn(bf16_hi(gw[i]), v1)));
+                                }
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    o[i] = pack_bf16x2(acc[c8 * 4 + i].x + bb[2 * i], acc[c8 * 4 + i].y + bb[2 * i + 1]);
+                            }
+                            st_shared_v4(stg + stage_off(static_cast<int>(lane), c), make_uint4(o[0], o[1], o[2], o[3]));
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(p.y + (m_w + 8 * j + pr) * p.N + ncol + pc * 8) =
+                                ld_shared_v4(stg + stage_off(8 * j + pr, pc));
+                        __syncwarp();
                     }
                 }
             }

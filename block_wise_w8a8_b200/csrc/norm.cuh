@@ -54,8 +54,6 @@
 namespace w8a8 {
 namespace norm {
 
-using quant::ld_shared_v4;
-
 constexpr int kStages = 6;
 constexpr int kGroups = 4;
 constexpr int kGroupWarps = 4;
@@ -90,13 +88,6 @@ static_assert(kStages >= kGroups && (2 * kStages) % kGroups == 0,
 __device__ __forceinline__ uint32_t chunk_off(int row, int c)
 {
     return static_cast<uint32_t>((c >> 3) * (128 * 64) + row * 64 + (((c & 7) ^ (row & 7)) << 3));
-}
-
-__device__ __forceinline__ void st_shared_v4(void *p, uint4 v)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x),
-                 "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank()

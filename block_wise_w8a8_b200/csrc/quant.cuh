@@ -111,14 +111,6 @@ static_assert(kQStages >= kQGroups, "every group needs a slot of its own");
 static_assert((2 * kQStages) % kQGroups == 0,
               "item it - 2 S of the ring must belong to the same group as item it");
 
-__device__ __forceinline__ uint4 ld_shared_v4(const void *p)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_u32(p)));
-    return v;
-}
 
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_blocks_kernel(const __grid_constant__ CUtensorMap tmX, int64_t K, int64_t nblocks,

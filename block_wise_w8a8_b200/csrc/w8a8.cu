@@ -26,7 +26,7 @@ constexpr int64_t kRowMaxK = 133120;
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
-    bool gemm_attr_set[4] = {false, false, false, false};
+    bool gemm_attr_set[5] = {false, false, false, false, false};
     bool quant_attr_set = false;
     bool norm_attr_set[4] = {false, false, false, false};
     int norm_max_clusters[norm::kMaxCluster + 1] = {};    // by cluster size, 0 = unknown
@@ -250,7 +250,8 @@ w8a8_status_t check_weight(const w8a8_weight_t *w, int64_t K)
 
 w8a8_status_t gemm_i8_impl(const int8_t *xq, const float *xs, int64_t M, int64_t K,
                            const w8a8_weight_t *w, const uint16_t *bias, uint16_t *y,
-                           cudaStream_t stream)
+                           cudaStream_t stream, const uint16_t *resid = nullptr,
+                           const uint16_t *gate = nullptr, int64_t gate_T = 1)
 {
     gemm::Params p{};
     p.M = M;
@@ -260,6 +261,11 @@ w8a8_status_t gemm_i8_impl(const int8_t *xq, const float *xs, int64_t M, int64_t
     p.ws = w->ws;
     p.bias = bias;
     p.y = y;
+    p.resid = resid;
+    p.gate = gate;
+    p.gate_T = gate_T;
+    if (gate != nullptr)
+        return launch_gemm<gemm::Mode::kI8Gated>(xq, w->wq, p, stream);
     return launch_gemm<gemm::Mode::kI8Scaled>(xq, w->wq, p, stream);
 }
 
@@ -587,6 +593,37 @@ w8a8_status_t w8a8_linear_prequant(const int8_t *xq, const float *xs, int64_t M,
     if (!aligned16(xq) || !aligned16(w->wq) || !aligned16(y) || (bias && !aligned16(bias)))
         return W8A8_ERR_ALIGNMENT;
     return gemm_i8_impl(xq, xs, M, K, w, bias, y, static_cast<cudaStream_t>(stream));
+}
+
+w8a8_status_t w8a8_linear_prequant_gated(const int8_t *xq, const float *xs, int64_t M, int64_t K,
+                                         const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                         const w8a8_bf16_t *resid, const w8a8_bf16_t *gate,
+                                         int64_t T, w8a8_bf16_t *y, void *stream)
+{
+    if (M < 0 || K < 0 || T <= 0)
+        return W8A8_ERR_INVALID_ARG;
+    W8A8_TRY(check_weight(w, K));
+    if (w->wq == nullptr)
+        return W8A8_ERR_INVALID_ARG;
+    if (M % T)
+        return W8A8_ERR_SHAPE;
+    if (M == 0 || w->N == 0)
+        return W8A8_OK;
+    if (!int8_shape_ok(M, K, w->N))
+        return W8A8_ERR_SHAPE;
+    W8A8_TRY(check_device_ptr(xq));
+    W8A8_TRY(check_device_ptr(xs));
+    W8A8_TRY(check_device_ptr(w->wq));
+    W8A8_TRY(check_device_ptr(w->ws));
+    W8A8_TRY(check_device_ptr(y));
+    W8A8_TRY(check_device_ptr(resid));
+    W8A8_TRY(check_device_ptr(gate));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    if (!aligned16(xq) || !aligned16(w->wq) || !aligned16(y) || (bias && !aligned16(bias)) ||
+        !aligned16(resid) || !aligned16(gate))
+        return W8A8_ERR_ALIGNMENT;
+    return gemm_i8_impl(xq, xs, M, K, w, bias, y, static_cast<cudaStream_t>(stream), resid, gate, T);
 }
 
 w8a8_status_t w8a8_bf16_linear(const w8a8_bf16_t *x, const w8a8_bf16_t *w,

@@ -197,6 +197,23 @@ W8A8_API w8a8_status_t w8a8_linear_prequant(const int8_t *xq, const float *xs, i
                                    const w8a8_weight_t *w, const w8a8_bf16_t *bias,
                                    w8a8_bf16_t *y, void *stream);
 
+/* w8a8_linear_prequant with the gated residual update fused into its epilogue
+ * (TurboT2VA paper, fused-operator paragraph: gated residual updates; the page gives no
+ * formula, this is the adaptive-norm block's form):
+ *     y[m,n] = bf16( fl( resid[m,n] + fl( gate[m/T, n] * v[m,n] ) ) )
+ * where v[m,n] is the FP32 value w8a8_linear_prequant would round to BF16 (bias
+ * included).  resid [M, N] BF16 may be y itself (an in-place update h += gate * linear);
+ * gate [M/T, N] BF16 must not overlap y.  T > 0 (else W8A8_ERR_INVALID_ARG) and dividing
+ * M (else W8A8_ERR_SHAPE); resid and gate 16-byte aligned device buffers; the rest as for
+ * w8a8_linear_prequant.  There is no BF16-path counterpart: shapes outside the INT8
+ * guard are rejected with W8A8_ERR_SHAPE and the caller applies the update itself. */
+W8A8_API w8a8_status_t w8a8_linear_prequant_gated(const int8_t *xq, const float *xs, int64_t M,
+                                                  int64_t K, const w8a8_weight_t *w,
+                                                  const w8a8_bf16_t *bias,
+                                                  const w8a8_bf16_t *resid,
+                                                  const w8a8_bf16_t *gate, int64_t T,
+                                                  w8a8_bf16_t *y, void *stream);
+
 /* The BF16 GEMM that the guard falls back to, callable directly:
  *   y[M, N] = bf16( sum_k x[m,k] w[n,k] (FP32 accumulation) + bias[n] ).
  *   Any M, K, N >= 0.  Uses tcgen05 tensor cores when K is a multiple of 8 and the
