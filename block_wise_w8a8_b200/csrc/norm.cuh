@@ -14,9 +14,9 @@
 // Work split.  A cluster of C <= 8 CTAs owns one 128-row strip at a time; CTA r handles
 // the strip's 128-column blocks kb = r, r + C, ...  (nb of them).  Each CTA streams its
 // blocks into a ring of six 32 KB shared-memory slots with 2-D TMA loads (two 64-column
-// boxes per block, 128-byte swizzle, no multicast).  When nb <= 6 the blocks stay in
-// their slots from the first pass to the second ("resident"), so x is read from HBM once;
-// otherwise every block is loaded twice (the second load normally hits L2).
+// boxes per block, 128-byte swizzle, no multicast), each block twice: once for the sums of
+// squares and once for the codes.  The second load comes about one strip later and is
+// served by L2 (a cluster has about two 1 MB strips in flight), so x crosses HBM once.
 //
 //   pass 1   each thread owns one row of a block and sums its squares in FP64.  The FP64
 //            operand is built from the BF16 bits with two integer operations, as |x| *
@@ -33,6 +33,14 @@
 //            8 (t % 16) .. +7.  2a normalises (and modulates), rounds to BF16, writes the
 //            values back into the slot and reduces the block's absmax; 2b forms the codes
 //            and stores them with 8-byte stores (a warp covers two full 128-byte rows).
+//
+// Pipelining.  Pass 1 runs one strip ahead of pass 2: the ring carries pass 1 of strip 0,
+// then, for each strip s, pass 1 of strip s + 1 followed by pass 2 of strip s.  The
+// exchange of strip s + 1 is sent while pass 2 of strip s runs and is awaited only after
+// pass 1 of strip s + 2, so its latency is hidden.  The exchange buffers (the CTA's group
+// partials, the C received partials, each group's rstd copy) are double-buffered by strip
+// parity; a CTA sends the partials of strip s + 1 only after all of its warps have read
+// those of strip s, which is what makes two buffers enough.
 //
 // Codes.  z = fl(y * fl(1/s) + 49152.5) lies in [2^15, 2^16), where the FP32 grid is
 // 2^-8, so byte 1 of z's bit pattern is the low byte of floor(z - 49152) = the code
@@ -59,7 +67,12 @@ constexpr int kGroups = 4;
 constexpr int kGroupWarps = 4;
 constexpr int kWarps = kGroups * kGroupWarps;   // consumer warps
 constexpr int kThreads = (kWarps + 1) * 32;     // + the TMA producer warp
-constexpr int kMaxCluster = 8;
+#ifndef W8A8_NORM_CLUSTER
+#define W8A8_NORM_CLUSTER 4
+#endif
+// CTAs per cluster (per strip).  Four: 37 clusters of one CTA per SM cover all 148 SMs of
+// a B200 (clusters of eight fit only 15 times), and each CTA gets K / 512 blocks a strip.
+constexpr int kMaxCluster = W8A8_NORM_CLUSTER;
 constexpr uint32_t kBlockBytes = 128 * 128 * 2;
 constexpr float kCodeMagic = 49152.5f;          // 1.5 * 2^15 + 1/2
 constexpr double kTwo256 = 1.157920892373162e77; // 2^256, exact
@@ -68,13 +81,13 @@ struct alignas(1024) Smem {
     uint16_t tile[kStages][128 * 128];         // two [128][64] boxes, 128-byte swizzle
     double part[2][kMaxCluster][128];          // [strip parity][source rank][row]
     double gpart[2][kGroups][128];             // [strip parity][group][row]
-    float rstd[kGroups][128];                  // each group's copy of the strip's rstd
+    float rstd[2][128];                        // [strip parity][row]
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t red_full[kGroups][2];
     uint64_t pdone[2];                         // all consumer warps wrote gpart
     uint64_t xready[2];                        // all C partials of every row arrived
-    uint64_t rready[kGroups];                  // the group's rstd copy is written
+    uint64_t rready;                           // the strip's rstd is written (all warps)
     alignas(16) uint32_t red[kGroups][2][kGroupWarps];
     int abort;
 };
@@ -176,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t K = p.K;
     const int64_t KB = K / 128;
     const int nb = KB > static_cast<int64_t>(rank) ? static_cast<int>((KB - 1 - rank) / C + 1) : 0;
-    const bool resident = nb <= kStages;
-    const int per_strip = resident ? nb : 2 * nb;
+    // strips this cluster handles: mb = cluster + s * nclusters, s = 0 .. ns - 1
+    const int64_t ns = cluster < p.MB ? (p.MB - 1 - cluster) / nclusters + 1 : 0;
     volatile int *abort = &sm.abort;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -187,34 +200,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < kGroups; ++g) {
             mbar_init(&sm.red_full[g][0], kGroupWarps);
             mbar_init(&sm.red_full[g][1], kGroupWarps);
-            mbar_init(&sm.rready[g], kGroupWarps);
         }
+        mbar_init(&sm.rready, kWarps);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.pdone[i], kWarps);
             mbar_init(&sm.xready[i], 1);
         }
         sm.abort = 0;
         fence_barrier_init();
+        // expect the partials of the first two strips (the sends may arrive first)
+        for (int64_t s = 0; s < 2 && s < ns; ++s)
+            mbar_arrive_expect_tx(&sm.xready[s], C * 128 * 8);
     }
     __syncthreads();
     cluster_barrier();      // every CTA's barriers are initialised before anything is sent
 
     if (warp == kWarps) {
         // ------------------------------------------------------------ TMA producer
-        // Items in load order: per strip, the CTA's nb blocks (resident), or its nb blocks
-        // for pass 1 followed by the same nb blocks again for pass 2.
+        // Items in load order: pass 1 of strip 0, then for each strip s pass 1 of strip
+        // s + 1 (if any) and pass 2 of strip s; each pass is the CTA's nb blocks in order.
         if (lane == 0 && nb > 0) {
             prefetch_tensormap(&tmX);
             uint32_t it = 0;
             bool ok = true;
-            for (int64_t mb = cluster; ok && mb < p.MB; mb += nclusters) {
-                for (int i = 0; i < per_strip; ++i, ++it) {
+            for (int64_t q = 0; ok && q <= 2 * ns; ++q) {
+                // q = 0: pass 1 of strip 0; odd q = 2 k - 1: pass 1 of strip k (there is
+                // none for k = ns); even q = 2 k: pass 2 of strip k - 1
+                const int64_t s = q == 0 ? 0 : ((q & 1) ? (q + 1) / 2 : q / 2 - 1);
+                if (s >= ns)
+                    continue;
+                const int64_t mb = cluster + s * nclusters;
+                for (int j = 0; j < nb; ++j, ++it) {
                     const uint32_t st = it % kStages, ph = (it / kStages) & 1;
                     if (!mbar_wait(&sm.empty[st], ph ^ 1, abort)) {
                         ok = false;
                         break;
                     }
-                    const int64_t kb = rank + static_cast<int64_t>(i < nb ? i : i - nb) * C;
+                    const int64_t kb = rank + static_cast<int64_t>(j) * C;
                     mbar_arrive_expect_tx(&sm.full[st], kBlockBytes);
                     tma_load_2d(sm.tile[st], &tmX, &sm.full[st], static_cast<int32_t>(kb * 128),
                                 static_cast<int32_t>(mb * 128));
@@ -236,38 +258,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------------- consumers
-    // Group g takes the strip's ring items it with it % 4 == g, in both passes.
+    // Group g takes the ring items it with it % 4 == g, in both passes.
     const int g = warp / kGroupWarps;
     const int gw = warp % kGroupWarps;
     const int gt = threadIdx.x % (kGroupWarps * 32);
     const int row0 = gt >> 4;              // pass 2: rows row0 + 8 j
     const int cc = gt & 15;                // pass 2: columns 8 cc .. 8 cc + 7
     const uint32_t o2 = static_cast<uint32_t>((cc >> 3) * (128 * 64) + row0 * 64 + (((cc & 7) ^ row0) << 3));
-    uint32_t base = 0;                     // ring items before this strip
+    uint32_t it_next = 0;                  // ring position of the next pass
     uint32_t gi = 0;                       // this group's pass-2 blocks so far
     bool dead = false;
-    int64_t sidx = 0;
-    for (int64_t mb = cluster; mb < p.MB; mb += nclusters, ++sidx, base += per_strip) {
-        const uint32_t sp = static_cast<uint32_t>(sidx & 1);
-        if (threadIdx.x == 0)
-            mbar_arrive_expect_tx(&sm.xready[sp], C * 128 * 8);
 
-        // pass 1: sum of squares of row gt over the group's blocks, four FP64 chains
+    // Waits for ring item it (after its slot's previous item, it - 6, has been released:
+    // a parity wait on full could otherwise match that older phase; item it - 12 belongs
+    // to this group and is released already, see the static_assert).
+    auto wait_item = [&](uint32_t it) -> bool {
+        const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+        bool ok = it < static_cast<uint32_t>(kStages) || mbar_wait(&sm.empty[st], ph ^ 1, abort);
+        ok = ok && mbar_wait(&sm.full[st], ph, abort);
+        return !__any_sync(0xFFFFFFFFu, !ok);
+    };
+
+    // Pass 1 of a strip: row gt's sum of squares over the group's blocks; writes the
+    // group's partial into gpart[sp].  Four FP64 chains, added in a fixed order.
+    auto pass1 = [&](uint32_t sp) -> bool {
+        const uint32_t base = it_next;
+        it_next += nb;
         double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        const int i0 = (g - static_cast<int>(base & 3) + 4) & 3;
-        for (int i = i0; i < nb; i += kGroups) {
+        for (int i = (g - static_cast<int>(base & 3) + 4) & 3; i < nb; i += kGroups) {
             const uint32_t it = base + i;
-            const uint32_t st = it % kStages, ph = (it / kStages) & 1;
-            // Slot st held item it - S before (another group's, possibly still in use):
-            // wait for its release first, so that the parity wait on full cannot match an
-            // older phase.  Item it - 2 S is known to be released (see the static_assert).
-            bool ok = it < static_cast<uint32_t>(kStages) || mbar_wait(&sm.empty[st], ph ^ 1, abort);
-            ok = ok && mbar_wait(&sm.full[st], ph, abort);
-            if (__any_sync(0xFFFFFFFFu, !ok)) {
-                dead = true;
-                break;
-            }
-            const uint16_t *tile = sm.tile[st];
+            if (!wait_item(it))
+                return false;
+            const uint16_t *tile = sm.tile[it % kStages];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 v = ld_shared_v4(tile + chunk_off(gt, c));
@@ -288,49 +310,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a2 = fma(d[6], d[6], a2);
                 a3 = fma(d[7], d[7], a3);
             }
-            if (!resident) {
-                // the sums depend on every value read: the slot is free again
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sm.empty[st]);
-            }
+            // the sums depend on every value read: the slot is free again
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.empty[it % kStages]);
         }
-        if (dead)
-            break;
-
-        // exchange: the CTA's partial of row gt (groups in order) to every CTA of the
-        // cluster; group g sends to ranks g, g + 4
         sm.gpart[sp][g][gt] = (a0 + a1) + (a2 + a3);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.pdone[sp]);
-        bool ok = mbar_wait(&sm.pdone[sp], static_cast<uint32_t>(sidx >> 1) & 1, abort);
-        if (__any_sync(0xFFFFFFFFu, !ok)) {
-            dead = true;
-            break;
-        }
+        return true;
+    };
+
+    // The CTA's partial of row gt for the strip of parity sp, sent to every CTA of the
+    // cluster; group g serves ranks g, g + 4.
+    auto send = [&](uint32_t sp) {
         const double cp = ((sm.gpart[sp][0][gt] + sm.gpart[sp][1][gt]) + sm.gpart[sp][2][gt]) +
                           sm.gpart[sp][3][gt];
         for (uint32_t c = static_cast<uint32_t>(g); c < C; c += kGroups)
             st_async_b64(map_to_rank(&sm.part[sp][rank][gt], c),
                          static_cast<uint64_t>(__double_as_longlong(cp)), map_to_rank(&sm.xready[sp], c));
-        ok = mbar_wait(&sm.xready[sp], static_cast<uint32_t>(sidx >> 1) & 1, abort);
-        if (__any_sync(0xFFFFFFFFu, !ok)) {
+    };
+
+    // pass 1 of strip 0 and its exchange
+    if (ns > 0) {
+        bool ok = pass1(0);
+        __syncwarp();
+        if (ok && lane == 0)
+            mbar_arrive(&sm.pdone[0]);
+        ok = ok && mbar_wait(&sm.pdone[0], 0, abort);
+        if (__any_sync(0xFFFFFFFFu, !ok))
+            dead = true;
+        else
+            send(0);
+    }
+    for (int64_t s = 0; s < ns && !dead; ++s) {
+        const int64_t mb = cluster + s * nclusters;
+        const uint32_t sp = static_cast<uint32_t>(s & 1);
+        const bool more = s + 1 < ns;
+        // pass 1 of the next strip
+        if (more && !pass1(sp ^ 1)) {
             dead = true;
             break;
         }
-        double tot = sm.part[sp][0][gt];
-        for (uint32_t c = 1; c < C; ++c)
-            tot += sm.part[sp][c][gt];
-        const double ss = kExactSq ? tot : tot * kTwo256;
-        const float r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(p.eps)));
-        sm.rstd[g][gt] = r;
-        if (p.rstd_out != nullptr && rank == 0 && g == 0)
-            p.rstd_out[mb * 128 + gt] = r;
+        // this strip's rstd, once per row: warp 0 of group g takes rows 32 g .. 32 g + 31,
+        // adding the row's C partials in rank order
+        if (gw == 0) {
+            const bool okx = mbar_wait(&sm.xready[sp], static_cast<uint32_t>(s >> 1) & 1, abort);
+            if (__any_sync(0xFFFFFFFFu, !okx)) {
+                dead = true;
+                break;
+            }
+            const int r = 32 * g + static_cast<int>(lane);
+            double tot = sm.part[sp][0][r];
+            for (uint32_t c = 1; c < C; ++c)
+                tot += sm.part[sp][c][r];
+            const double ss = kExactSq ? tot : tot * kTwo256;
+            const float rv = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(p.eps)));
+            sm.rstd[sp][r] = rv;
+            if (p.rstd_out != nullptr && rank == 0)
+                p.rstd_out[mb * 128 + r] = rv;
+            if (threadIdx.x == 0 && s + 2 < ns)
+                mbar_arrive_expect_tx(&sm.xready[sp], C * 128 * 8);
+        }
+        // pdone of the next strip: its group partials are written and this strip's
+        // received partials have been read (so the next sends may overwrite them)
         __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.rready[g]);
-        ok = mbar_wait(&sm.rready[g], static_cast<uint32_t>(sidx & 1), abort);
+        if (lane == 0) {
+            if (more)
+                mbar_arrive(&sm.pdone[sp ^ 1]);
+            mbar_arrive(&sm.rready);
+        }
+        bool ok = mbar_wait(&sm.rready, sp, abort);
         if (__any_sync(0xFFFFFFFFu, !ok)) {
             dead = true;
             break;
@@ -338,26 +386,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         float rs[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            rs[j] = sm.rstd[g][row0 + 8 * j];
-        const int64_t bm = kMod ? (mb * 128) / p.T : 0;     // the strip's modulation row
+            rs[j] = sm.rstd[sp][row0 + 8 * j];
+        if (more) {
+            ok = mbar_wait(&sm.pdone[sp ^ 1], static_cast<uint32_t>((s + 1) >> 1) & 1, abort);
+            if (__any_sync(0xFFFFFFFFu, !ok)) {
+                dead = true;
+                break;
+            }
+            send(sp ^ 1);
+        }
 
         // pass 2: normalise (modulate), round to BF16, quantize each of the group's blocks
-        const int first = resident ? i0 : nb + ((g - static_cast<int>((base + nb) & 3) + 4) & 3);
-        const int last = resident ? nb : 2 * nb;
-        for (int i = first; i < last; i += kGroups, ++gi) {
-            const int j = resident ? i : i - nb;
+        const int64_t bm = kMod ? (mb * 128) / p.T : 0;     // the strip's modulation row
+        const uint32_t base = it_next;
+        it_next += nb;
+        for (int i = (g - static_cast<int>(base & 3) + 4) & 3; i < nb; i += kGroups, ++gi) {
             const uint32_t it = base + i;
-            const uint32_t st = it % kStages, ph = (it / kStages) & 1;
-            if (!resident) {
-                bool ok2 = it < static_cast<uint32_t>(kStages) || mbar_wait(&sm.empty[st], ph ^ 1, abort);
-                ok2 = ok2 && mbar_wait(&sm.full[st], ph, abort);
-                if (__any_sync(0xFFFFFFFFu, !ok2)) {
-                    dead = true;
-                    break;
-                }
-            }
-            const int64_t kb = rank + static_cast<int64_t>(j) * C;
+            const int64_t kb = rank + static_cast<int64_t>(i) * C;
             const int64_t col = kb * 128 + cc * 8;
+            // the per-column factors are loaded before the wait for the block
             float gm[8], am[8], sh[8];
             if (p.gamma != nullptr) {
                 unpack8(__ldg(reinterpret_cast<const uint4 *>(p.gamma + col)), gm);
@@ -373,7 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 8; ++e)
                     am[e] = __fadd_rn(1.0f, am[e]);
             }
-            uint16_t *tile = sm.tile[st] + o2;
+            if (!wait_item(it)) {
+                dead = true;
+                break;
+            }
+            uint16_t *tile = sm.tile[it % kStages] + o2;
 
             // 2a: y = bf16(...) written back in place; the block's absmax
             uint32_t m2 = 0;
@@ -382,15 +433,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint4 v = ld_shared_v4(tile + jj * 512);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                 uint32_t o[4];
+                const float2 r2 = make_float2(rs[jj], rs[jj]);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    float n0 = __fmul_rn(__fmul_rn(bf16_lo(w[k]), rs[jj]), gm[2 * k]);
-                    float n1 = __fmul_rn(__fmul_rn(bf16_hi(w[k]), rs[jj]), gm[2 * k + 1]);
+                    float2 n = __fmul2_rn(make_float2(bf16_lo(w[k]), bf16_hi(w[k])), r2);
+                    n = __fmul2_rn(n, make_float2(gm[2 * k], gm[2 * k + 1]));
                     if (kMod) {
-                        n0 = __fadd_rn(__fmul_rn(n0, am[2 * k]), sh[2 * k]);
-                        n1 = __fadd_rn(__fmul_rn(n1, am[2 * k + 1]), sh[2 * k + 1]);
+                        // the shift is added with the scalar __fadd_rn, which is never
+                        // contracted with the product into a fused multiply-add (the
+                        // packed add gives no such guarantee); the definition rounds twice
+                        n = __fmul2_rn(n, make_float2(am[2 * k], am[2 * k + 1]));
+                        n.x = __fadd_rn(n.x, sh[2 * k]);
+                        n.y = __fadd_rn(n.y, sh[2 * k + 1]);
                     }
-                    o[k] = pack_bf16x2(n0, n1);
+                    o[k] = pack_bf16x2(n.x, n.y);
                 }
                 st_shared_v4(tile + jj * 512, make_uint4(o[0], o[1], o[2], o[3]));
                 m2 = quant::absmax8_bits(o, m2);
@@ -419,6 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // 2b: codes from z = y * (1/s) + 49152.5 (byte 1), fraction byte 0 flags a tie
             int8_t *qb = p.q + (mb * 128 + row0) * K + col;
+            const float2 rc2 = make_float2(rc, rc);
+            const float2 magic2 = make_float2(kCodeMagic, kCodeMagic);
             uint32_t flagged = 0;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
@@ -427,9 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t pr[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint32_t t0 = __float_as_uint(__fmaf_rn(bf16_lo(w[k]), rc, kCodeMagic));
-                    const uint32_t t1 = __float_as_uint(__fmaf_rn(bf16_hi(w[k]), rc, kCodeMagic));
-                    pr[k] = __byte_perm(t0, t1, 0x5410);      // frac0 code0 frac1 code1
+                    const float2 z = __ffma2_rn(make_float2(bf16_lo(w[k]), bf16_hi(w[k])), rc2, magic2);
+                    pr[k] = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x5410);  // frac0 code0 frac1 code1
                 }
                 *reinterpret_cast<uint2 *>(qb + static_cast<int64_t>(jj) * 8 * K) =
                     make_uint2(__byte_perm(pr[0], pr[1], 0x7531), __byte_perm(pr[2], pr[3], 0x7531));
@@ -457,10 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every lane is done with the slot
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm.empty[st]);
+                mbar_arrive(&sm.empty[it % kStages]);
         }
-        if (dead)
-            break;
     }
     __syncwarp();
     cluster_barrier();      // no CTA leaves while a peer may still send to it
