@@ -95,6 +95,10 @@ __device__ __forceinline__ uint32_t stage_off(int r, int c)
 struct Params {
     int64_t M, N, K;
     int32_t num_tm, num_tn, num_tiles, kslices;
+    // Work units: units 0 .. num_full - 1 are whole tiles (in tile order); the remaining
+    // tiles are each split into two 128-column halves, units num_full + 2 i + h.  The
+    // host splits only the scaled modes' last, partial round of tiles.
+    int32_t num_full, num_units;
     const float *xs;          // [M/128, K/128] (INT8 modes)
     const float *ws;          // [N/128, K/128] (INT8 modes)
     const uint16_t *bias;     // [N] BF16 or null
@@ -116,6 +120,19 @@ __device__ __forceinline__ void tile_coords(int t, int num_tm, int num_tn, int &
     const int local = t - group * per_group;
     tm = first + local % gsz;
     tn = local / gsz;
+}
+
+// The tile of work unit u and which 128-column half of it (-1: the whole tile).
+__device__ __forceinline__ void unit_coords(int u, const Params &p, int &tm, int &tn, int &hs)
+{
+    if (u < p.num_full) {
+        tile_coords(u, p.num_tm, p.num_tn, tm, tn);
+        hs = -1;
+    } else {
+        const int v = u - p.num_full;
+        tile_coords(p.num_full + (v >> 1), p.num_tm, p.num_tn, tm, tn);
+        hs = v & 1;
+    }
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p)
@@ -220,9 +237,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-                int tm, tn;
-                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+            for (int t = blockIdx.x; ok && t < p.num_units; t += gridDim.x) {
+                int tm, tn, hs;
+                unit_coords(t, p, tm, tn, hs);
                 for (int ks = 0; ks < p.kslices; ++ks, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, abort)) {
@@ -245,10 +262,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = kInt8 ? idesc_i8_s32(BM, BN) : idesc_bf16_f32(BM, BN);
+            const uint32_t idesc_full = kInt8 ? idesc_i8_s32(BM, BN) : idesc_bf16_f32(BM, BN);
+            const uint32_t idesc_half = idesc_i8_s32(BM, BN / 2);
             uint32_t it = 0, acc_i = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+            for (int t = blockIdx.x; ok && t < p.num_units; t += gridDim.x) {
+                int tm, tn, hs;
+                unit_coords(t, p, tm, tn, hs);
+                // a half unit multiplies by rows 128 hs .. 128 hs + 127 of the B tile (16 KB
+                // further in shared memory) into the first 128 accumulator columns
+                const uint32_t idesc = hs < 0 ? idesc_full : idesc_half;
+                const uint64_t b_off = hs < 0 ? 0 : static_cast<uint64_t>(hs) * ((BN / 2) * 128 / 16);
                 uint32_t buf = acc_i & 1;
                 if (!kPerKb) {
                     if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
@@ -273,7 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     const uint32_t d = tmem + buf * BN;
                     const uint64_t ad = umma_desc_sw128(smem_u32(sm.a[s]));
-                    const uint64_t bd = umma_desc_sw128(smem_u32(sm.b[s]));
+                    const uint64_t bd = umma_desc_sw128(smem_u32(sm.b[s])) + b_off;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         // each MMA consumes 32 bytes of K: advance start address by 32 B
@@ -336,9 +360,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (kScaled) {
             const int KB = static_cast<int>(p.K / 128);
             constexpr int kEpiThreads = NUM_EPI_WARPS * 32;
-            if (static_cast<int>(blockIdx.x) < p.num_tiles) {
-                int tm, tn;
-                tile_coords(blockIdx.x, p.num_tm, p.num_tn, tm, tn);
+            if (static_cast<int>(blockIdx.x) < p.num_units) {
+                int tm, tn, hs;
+                unit_coords(blockIdx.x, p, tm, tn, hs);
                 scales_fetch(sm.sx[0], sm.sw[0], p, tm, tn, etid, kEpiThreads);
                 cp_async_wait_all();
             }
@@ -346,23 +370,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // No named barriers here: every wait of the epilogue is a bounded mbarrier
             // wait, so an abort can never leave part of the warps parked in bar.sync.
             int tile_iter = 0;
-            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tile_iter) {
-                int tm, tn;
-                tile_coords(t, p.num_tm, p.num_tn, tm, tn);
+            for (int t = blockIdx.x; t < p.num_units; t += gridDim.x, ++tile_iter) {
+                int tm, tn, hs;
+                unit_coords(t, p, tm, tn, hs);
+                // A half unit's sums sit in the first 128 accumulator columns: warpgroup 1
+                // takes them (for output half hs); warpgroup 2 only keeps step with the
+                // accumulator barriers.
+                const bool active = hs < 0 || half == 0;
+                const int hcol = hs < 0 ? half : hs;
                 const int sb = tile_iter & 1;
                 // the scales of this tile were copied by all epilogue threads during the
                 // previous tile
                 if (!mbar_wait(&sm.sready[sb], (tile_iter >> 1) & 1, abort))
                     break;
                 const int tnext = t + gridDim.x;
-                if (tnext < p.num_tiles) {
-                    int tm2, tn2;
-                    tile_coords(tnext, p.num_tm, p.num_tn, tm2, tn2);
+                if (tnext < p.num_units) {
+                    int tm2, tn2, hs2;
+                    unit_coords(tnext, p, tm2, tn2, hs2);
                     scales_fetch(sm.sx[sb ^ 1], sm.sw[sb ^ 1], p, tm2, tn2, etid, kEpiThreads);
                 }
-                if (kMode == Mode::kI8Gated) {
+                if (kMode == Mode::kI8Gated && active) {
                     const int64_t pm = static_cast<int64_t>(tm) * BM + row;
-                    const int64_t pn = static_cast<int64_t>(tn) * BN + half * 128;
+                    const int64_t pn = static_cast<int64_t>(tn) * BN + hcol * 128;
                     if (pn < p.N) {
                         prefetch_l2(p.resid + pm * p.N + pn);
                         prefetch_l2(p.resid + pm * p.N + pn + 64);
@@ -373,36 +402,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int j = 0; j < 64; ++j)
                     acc[j] = make_float2(0.0f, 0.0f);
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
-                    const uint32_t buf = acc_i & 1;
-                    if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const float sc = sm.sx[sb][kb] * sm.sw[sb][half][kb];   // FP32 scale product
-                    const float2 sc2 = make_float2(sc, sc);
-                    const float2 nmg = make_float2(-kAccInitF, -kAccInitF);
-                    const uint32_t tb = lane_base + buf * BN;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t r[16];
-                        tmem_ld16(tb + c * 16, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float2 v = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                            v = __fadd2_rn(v, nmg);                         // float(P), exact
-                            acc[c * 8 + j] = __ffma2_rn(v, sc2, acc[c * 8 + j]);
+                if (active) {
+                    const uint32_t lb = hs < 0 ? lane_base : lane_base - half * 128;
+                    for (int kb = 0; kb < KB; ++kb) {
+                        const uint32_t buf = acc_i & 1;
+                        if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                            ok = false;
+                            break;
                         }
-                        tmem_st16(tb + c * 16, fill);
+                        tc_fence_after();
+                        const float sc = sm.sx[sb][kb] * sm.sw[sb][hcol][kb];   // FP32 scale product
+                        const float2 sc2 = make_float2(sc, sc);
+                        const float2 nmg = make_float2(-kAccInitF, -kAccInitF);
+                        const uint32_t tb = lb + buf * BN;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            uint32_t r[16];
+                            tmem_ld16(tb + c * 16, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                float2 v = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                                v = __fadd2_rn(v, nmg);                     // float(P), exact
+                                acc[c * 8 + j] = __ffma2_rn(v, sc2, acc[c * 8 + j]);
+                            }
+                            tmem_st16(tb + c * 16, fill);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&sm.tempty[buf]);
+                        ++acc_i;
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&sm.tempty[buf]);
-                    ++acc_i;
+                } else {
+                    // warpgroup 2 during a half unit: keep step with the accumulator barriers
+                    for (int kb = 0; kb < KB; ++kb) {
+                        const uint32_t buf = acc_i & 1;
+                        if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&sm.tempty[buf]);
+                        ++acc_i;
+                    }
                 }
                 if (!ok)
                     break;
@@ -415,9 +462,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // row segments, 8 rows per instruction (8 cache lines instead of 32).  The
                 // gated mode reads the residual the same way in reverse.
                 const int64_t m = static_cast<int64_t>(tm) * BM + row;
-                const int64_t n0 = static_cast<int64_t>(tn) * BN + half * 128;
+                const int64_t n0 = static_cast<int64_t>(tn) * BN + hcol * 128;
                 const int64_t m_w = m - static_cast<int64_t>(lane);
-                if (n0 < p.N) {
+                if (active && n0 < p.N) {
                     uint8_t *stg = sm.stage[ew];
                     const int pr = static_cast<int>(lane >> 2), pc = static_cast<int>(lane & 3);
                     const uint16_t *gp = kMode == Mode::kI8Gated ? p.gate + (m / p.gate_T) * p.N + n0 : nullptr;

@@ -180,7 +180,20 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
             g_dev[dev].gemm_attr_set[static_cast<int>(kMode)] = true;
         }
     }
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, g_dev[dev].sms));
+    // Work units: whole tiles, except that in the scaled modes a last, partial round of
+    // tiles is split into 128-column halves when they all fit in one round (a half takes
+    // about half a tile's time: the epilogue, the bottleneck, does half the work).
+    const int sms = g_dev[dev].sms;
+    p.num_full = p.num_tiles;
+    p.num_units = p.num_tiles;
+    if (kMode == gemm::Mode::kI8Scaled || kMode == gemm::Mode::kI8Gated) {
+        const int tail = p.num_tiles % sms;
+        if (tail > 0 && 2 * tail <= sms) {
+            p.num_full = p.num_tiles - tail;
+            p.num_units = p.num_full + 2 * tail;
+        }
+    }
+    const int grid = std::min(p.num_units, sms);
     kern<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, stream>>>(ta, tb, p);
     return launch_status();
 }
