@@ -42,14 +42,9 @@
 // parity; a CTA sends the partials of strip s + 1 only after all of its warps have read
 // those of strip s, which is what makes two buffers enough.
 //
-// Codes.  z = fl(y * fl(1/s) + 49152.5) lies in [2^15, 2^16), where the FP32 grid is
-// 2^-8, so byte 1 of z's bit pattern is the low byte of floor(z - 49152) = the code
-// (two's complement) and byte 0 is the fraction of z on that grid.  |z - 49152.5 -
-// fl32(y / s)| < 2^-9 + 2^-16, so unless the fraction byte is 0 (z within 2^-9 of an
-// integer, i.e. y / s near a half-integer) floor(z - 49152) = rne(fl32(y / s)).  Entries
-// with fraction byte 0 (about 0.4%), and all entries of a block whose 1/s overflows, are
-// recomputed with the IEEE division, so the codes equal those of the definition bit for
-// bit.  The clamp cannot fire on the fast path (|y / s| <= 127 (1 + 2^-22)).
+// Codes as in quant.cuh (quant::codes8): one FFMA onto the 2^-8 grid above 49152.5, the
+// code in byte 1, and the 0.4% of values whose fraction byte flags a possible tie
+// recomputed with the IEEE division, so the codes equal the definition's bit for bit.
 //
 // Every wait is a bounded mbarrier wait.  The kernel's only unbounded waits are the two
 // cluster barriers at its start and end, which every thread reaches after finitely many
@@ -74,7 +69,6 @@ constexpr int kThreads = (kWarps + 1) * 32;     // + the TMA producer warp
 // a B200 (clusters of eight fit only 15 times), and each CTA gets K / 512 blocks a strip.
 constexpr int kMaxCluster = W8A8_NORM_CLUSTER;
 constexpr uint32_t kBlockBytes = 128 * 128 * 2;
-constexpr float kCodeMagic = 49152.5f;          // 1.5 * 2^15 + 1/2
 constexpr double kTwo256 = 1.157920892373162e77; // 2^256, exact
 
 struct alignas(1024) Smem {
@@ -473,43 +467,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (gt == 0)
                 p.s[mb * KB + kb] = sc;
 
-            // 2b: codes from z = y * (1/s) + 49152.5 (byte 1), fraction byte 0 flags a tie
+            // 2b: the codes (quant::codes8: z = y * (1/s) + 49152.5), ties re-done exactly
             int8_t *qb = p.q + (mb * 128 + row0) * K + col;
             const float2 rc2 = make_float2(rc, rc);
-            const float2 magic2 = make_float2(kCodeMagic, kCodeMagic);
             uint32_t flagged = 0;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
                 const uint4 v = ld_shared_v4(tile + jj * 512);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t pr[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 z = __ffma2_rn(make_float2(bf16_lo(w[k]), bf16_hi(w[k])), rc2, magic2);
-                    pr[k] = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x5410);  // frac0 code0 frac1 code1
-                }
-                *reinterpret_cast<uint2 *>(qb + static_cast<int64_t>(jj) * 8 * K) =
-                    make_uint2(__byte_perm(pr[0], pr[1], 0x7531), __byte_perm(pr[2], pr[3], 0x7531));
-                const uint32_t fr = __vminu2(__vminu2(pr[0] & 0x00FF00FFu, pr[1] & 0x00FF00FFu),
-                                             __vminu2(pr[2] & 0x00FF00FFu, pr[3] & 0x00FF00FFu));
-                flagged |= ((fr & 0xFFFFu) == 0 || (fr >> 16) == 0) ? (1u << jj) : 0u;
+                bool tie;
+                // streaming store: the codes are not read again by this kernel
+                __stcs(reinterpret_cast<uint2 *>(qb + static_cast<int64_t>(jj) * 8 * K), quant::codes8(w, rc2, tie));
+                flagged |= tie ? (1u << jj) : 0u;
             }
-            // Entries whose fraction byte is 0, and every entry of a block whose 1/s
-            // overflows (s below about 2^-128), take their code from the IEEE division;
-            // the byte stores land after the 8-byte stores above (same thread, same address).
+            // Chunks with a value near a half-integer are re-coded exactly, every chunk of a
+            // block whose 1/s overflows (s below about 2^-128) by division; the later
+            // 8-byte store to the same address, by the same thread, wins.
             const bool all_exact = !(rc <= 3.0e38f);
             if (all_exact)
                 flagged = 0xFFFFu;
             while (flagged != 0) {
                 const int jj = __ffs(flagged) - 1;
                 flagged &= flagged - 1;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float y = __uint_as_float(static_cast<uint32_t>(tile[jj * 512 + e]) << 16);
-                    const uint32_t t = __float_as_uint(__fmaf_rn(y, rc, kCodeMagic));
-                    if (all_exact || (t & 0xFFu) == 0)
-                        qb[static_cast<int64_t>(jj) * 8 * K + e] = static_cast<int8_t>(quant::code_exact(y, sc));
-                }
+                const uint4 v = ld_shared_v4(tile + jj * 512);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                __stcs(reinterpret_cast<uint2 *>(qb + static_cast<int64_t>(jj) * 8 * K),
+                       all_exact ? quant::codes8_division(w, sc) : quant::codes8_exact(w, rc, sc));
             }
             // every lane is done with the slot
             __syncwarp();

@@ -15,6 +15,15 @@
 // division itself, so the codes equal those of the definition bit for bit.  The clamp
 // cannot fire on the fast path (|y| <= 127 * (1 + 2^-22) rounds to at most 127); the
 // exact path keeps it.
+//
+// codes8 (used after RMSNorm, norm.cuh) trades that band for fewer instructions:
+// z = fl(v * fl(1/s) + 49152.5) lies in [2^15, 2^16), where the FP32 grid is 2^-8, so byte 1
+// of z's bit pattern is the low byte of floor(z - 49152), the code in two's complement, and
+// byte 0 is the fraction of z on that grid.  |z - 49152.5 - fl32(v / s)| < 2^-9 + 2^-16, so
+// unless the fraction byte is 0 (z within 2^-9 of an integer) floor(z - 49152) equals
+// rne(fl32(v / s)).  A chunk holding such a value (about 3% of 8-value chunks) is re-coded
+// with codes8_exact.  In the standalone quantizers that re-coding costs more than codes8
+// saves (measured), so they keep quantize8_fast.
 #pragma once
 
 #include "common.cuh"
@@ -24,6 +33,7 @@ namespace quant {
 
 constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23
 constexpr float kTieBand = 0.5f - 1.0f / 16384.0f;     // entries with |y - rne(y)| >= this
+constexpr float kCodeMagic = 49152.5f;                 // 1.5 * 2^15 + 1/2 (codes8)
 
 // Exact code of one value: IEEE quotient by the stored scale, rint (half to even), clamp.
 __device__ __forceinline__ uint32_t code_exact(float v, float sc)
@@ -61,6 +71,61 @@ __device__ __forceinline__ uint2 quantize8_fast(const uint32_t (&w)[4], float rc
     out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
     out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
     return out;
+}
+
+// Codes of 8 BF16 values (4 packed words, element 2i in the low half of w[i]) as 8
+// bytes, through z = fl(v * rc + 49152.5) (see above).  `tie` is set when some value's
+// fraction byte is 0: the chunk must then be re-coded with codes8_exact.
+__device__ __forceinline__ uint2 codes8(const uint32_t (&w)[4], float2 rc2, bool &tie)
+{
+    const float2 mg = make_float2(kCodeMagic, kCodeMagic);
+    uint32_t pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 z = __ffma2_rn(make_float2(bf16_lo(w[i]), bf16_hi(w[i])), rc2, mg);
+        pr[i] = __byte_perm(__float_as_uint(z.x), __float_as_uint(z.y), 0x5410);  // frac code frac code
+    }
+    const uint32_t fr = __vminu2(__vminu2(pr[0] & 0x00FF00FFu, pr[1] & 0x00FF00FFu),
+                                 __vminu2(pr[2] & 0x00FF00FFu, pr[3] & 0x00FF00FFu));
+    tie = (fr & 0xFFFFu) == 0 || (fr >> 16) == 0;
+    return make_uint2(__byte_perm(pr[0], pr[1], 0x7531), __byte_perm(pr[2], pr[3], 0x7531));
+}
+
+// Exact codes of 8 BF16 values, for a chunk that codes8 flagged: quantize8_fast's
+// arithmetic (a band about 30 times narrower than codes8's), and the IEEE division for
+// the values inside it.
+__device__ __forceinline__ uint2 codes8_exact(const uint32_t (&w)[4], float rc, float sc)
+{
+    const float2 r2 = make_float2(rc, rc);
+    const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+    const float2 nmg = make_float2(-kRoundMagic, -kRoundMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    uint32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 v = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
+        const float2 y = __fmul2_rn(v, r2);          // ~ v / s
+        const float2 tt = __fadd2_rn(y, mg);         // 1.5 * 2^23 + rne(y): low byte = code
+        const float2 n = __fadd2_rn(tt, nmg);        // rne(y), exact
+        const float2 d = __ffma2_rn(n, neg1, y);     // y - rne(y), exact
+        t[2 * i] = fabsf(d.x) >= kTieBand ? code_exact(v.x, sc) : __float_as_uint(tt.x);
+        t[2 * i + 1] = fabsf(d.y) >= kTieBand ? code_exact(v.y, sc) : __float_as_uint(tt.y);
+    }
+    return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
+}
+
+// Codes of 8 values whose 1/s overflowed (s below about 2^-128): the IEEE division for all.
+__device__ __forceinline__ uint2 codes8_division(const uint32_t (&w)[4], float sc)
+{
+    uint32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        t[2 * i] = code_exact(bf16_lo(w[i]), sc);
+        t[2 * i + 1] = code_exact(bf16_hi(w[i]), sc);
+    }
+    return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
 }
 
 // Largest |BF16| among 8 values, as a BF16 magnitude pattern in the low 16 bits
