@@ -115,8 +115,8 @@ W8A8_API w8a8_status_t w8a8_quantize_act(const w8a8_bf16_t *x, int64_t M, int64_
  *   xs [M/128, K/128] FP32, and rstd_out [M] FP32 when not NULL.
  *   M, K multiples of 128 (else W8A8_ERR_SHAPE; M == 0 is a no-op), eps >= 0 and finite
  *   (else W8A8_ERR_INVALID_ARG); x, gamma, xq 16-byte aligned, xs and rstd_out 4-byte
- *   aligned.  Reads x once from HBM when K <= 6144 (the strip's blocks stay on chip
- *   between the two passes), twice (the second from L2) above that. */
+ *   aligned.  Each block of x is loaded twice, once for the row sums and once for the
+ *   codes; the second load is mostly served by L2. */
 W8A8_API w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
                                         float eps, int64_t M, int64_t K, int8_t *xq,
                                         float *xs, float *rstd_out, void *stream);
