@@ -135,6 +135,43 @@ __device__ __forceinline__ void unit_coords(int u, const Params &p, int &tm, int
     }
 }
 
+// The GEMM's bounded mbarrier wait.  Its try_wait carries a suspend-time hint, so a
+// waiting thread sleeps in hardware until the phase completes instead of re-polling:
+// the TMA producer and the MMA thread share SM sub-partitions with epilogue warps, and
+// their polling took issue slots from them.  Otherwise as mbar_wait: false after a
+// timeout (recorded, *abort raised) or once another thread has raised *abort.
+__device__ __forceinline__ bool try_wait_sleep(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(1000000)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool gemm_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    const uint32_t b = smem_u32(bar);
+    if (try_wait_sleep(b, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (try_wait_sleep(b, parity))
+            return true;
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            *abort = 1;
+            record_device_error(1);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void prefetch_l2(const void *p)
 {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -242,7 +279,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 unit_coords(t, p, tm, tn, hs);
                 for (int ks = 0; ks < p.kslices; ++ks, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1, abort)) {
+                    if (!gemm_wait(&sm.empty[s], ph ^ 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -275,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint64_t b_off = hs < 0 ? 0 : static_cast<uint64_t>(hs) * ((BN / 2) * 128 / 16);
                 uint32_t buf = acc_i & 1;
                 if (!kPerKb) {
-                    if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
+                    if (!gemm_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -283,16 +320,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 for (int ks = 0; ks < p.kslices; ++ks, ++it) {
                     const uint32_t s = it % STAGES, ph = (it / STAGES) & 1;
+                    // the stage first: it is normally loaded long before the accumulator
+                    // comes back, so the MMAs go out as soon as the epilogue releases it
+                    if (!gemm_wait(&sm.full[s], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
                     if (kPerKb) {
                         buf = acc_i & 1;
-                        if (!mbar_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
+                        if (!gemm_wait(&sm.tempty[buf], (acc_i >> 1) & 1, abort)) {
                             ok = false;
                             break;
                         }
-                    }
-                    if (!mbar_wait(&sm.full[s], ph, abort)) {
-                        ok = false;
-                        break;
                     }
                     tc_fence_after();
                     const uint32_t d = tmem + buf * BN;
@@ -381,7 +420,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int sb = tile_iter & 1;
                 // the scales of this tile were copied by all epilogue threads during the
                 // previous tile
-                if (!mbar_wait(&sm.sready[sb], (tile_iter >> 1) & 1, abort))
+                if (!gemm_wait(&sm.sready[sb], (tile_iter >> 1) & 1, abort))
                     break;
                 const int tnext = t + gridDim.x;
                 if (tnext < p.num_units) {
@@ -406,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t lb = hs < 0 ? lane_base : lane_base - half * 128;
                     for (int kb = 0; kb < KB; ++kb) {
                         const uint32_t buf = acc_i & 1;
-                        if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                        if (!gemm_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
                             ok = false;
                             break;
                         }
@@ -439,7 +478,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     // warpgroup 2 during a half unit: keep step with the accumulator barriers
                     for (int kb = 0; kb < KB; ++kb) {
                         const uint32_t buf = acc_i & 1;
-                        if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                        if (!gemm_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
                             ok = false;
                             break;
                         }
@@ -528,7 +567,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     const uint32_t buf = acc_i & 1;
-                    if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
+                    if (!gemm_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -567,7 +606,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 int tm, tn;
                 tile_coords(t, p.num_tm, p.num_tn, tm, tn);
                 const uint32_t buf = acc_i & 1;
-                if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
+                if (!gemm_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
                     break;
                 tc_fence_after();
                 const int64_t m = static_cast<int64_t>(tm) * BM + row;
@@ -627,7 +666,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 int tm, tn;
                 tile_coords(t, p.num_tm, p.num_tn, tm, tn);
                 const uint32_t buf = acc_i & 1;
-                if (!mbar_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
+                if (!gemm_wait(&sm.tfull[buf], (acc_i >> 1) & 1, abort))
                     break;
                 tc_fence_after();
                 const int64_t m = static_cast<int64_t>(tm) * BM + row;
