@@ -52,6 +52,9 @@ _SIGS = {
     "w8a8_linear": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                     ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
+    "w8a8_linear_host": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(_Weight),
+                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                         ctypes.c_int64, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
     "w8a8_linear_noalloc": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                             ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p,
                             ctypes.POINTER(ctypes.c_int), ctypes.c_void_p],
@@ -85,6 +88,10 @@ def lib():
             fn.restype = ctypes.c_int
         L.w8a8_linear_workspace_bytes.argtypes = [ctypes.c_int64] * 3
         L.w8a8_linear_workspace_bytes.restype = ctypes.c_size_t
+        L.w8a8_linear_host_workspace_bytes.argtypes = [ctypes.c_int64] * 4
+        L.w8a8_linear_host_workspace_bytes.restype = ctypes.c_size_t
+        L.w8a8_linear_host_chunk_rows.argtypes = [ctypes.c_int64] * 2
+        L.w8a8_linear_host_chunk_rows.restype = ctypes.c_int64
         L.w8a8_device_error.argtypes = []
         L.w8a8_device_error.restype = ctypes.c_int
         L.w8a8_last_cuda_error.argtypes = []
@@ -260,6 +267,41 @@ def linear(x, weight, bias=None, out=None, workspace=None, return_path=False):
     _check("w8a8_linear", lib().w8a8_linear(
         _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
         0 if workspace is None else workspace.numel(), ctypes.byref(path), _stream(dev)))
+    return (out, path.value) if return_path else out
+
+
+def linear_host_workspace_bytes(M, K, N, chunk_rows=0):
+    return int(lib().w8a8_linear_host_workspace_bytes(M, K, N, chunk_rows))
+
+
+def linear_host(x, weight, bias=None, out=None, workspace=None, chunk_rows=0, return_path=False):
+    """w8a8_linear on host buffers: x [..., K] BF16 and the output in CPU memory (pinned
+    memory lets the copies overlap with the compute).  The rows stream through the GPU in
+    chunks; the result equals linear() on a device copy of x.  The work is enqueued on the
+    weight device's current stream, which completes only after the output has landed in
+    host memory."""
+    if not isinstance(x, torch.Tensor) or x.device.type != "cpu":
+        raise ValueError("x must be a CPU tensor (use linear() for device tensors)")
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous torch.bfloat16 tensor")
+    if bias is not None:
+        _need(bias, torch.bfloat16, "bias")
+    K = x.shape[-1]
+    M = math.prod(x.shape[:-1])
+    N = weight.N
+    dev = weight.w.device
+    if out is None:
+        out = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, pin_memory=True)
+    elif out.device.type != "cpu" or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU torch.bfloat16 tensor")
+    need = linear_host_workspace_bytes(M, K, N, chunk_rows)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    path = ctypes.c_int(-1)
+    _check("w8a8_linear_host", lib().w8a8_linear_host(
+        _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), chunk_rows, ctypes.byref(path),
+        _stream(dev)))
     return (out, path.value) if return_path else out
 
 

@@ -5,6 +5,7 @@
 // enqueued on the caller's stream; nothing is allocated.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/w8a8.h"
@@ -434,6 +435,63 @@ w8a8_status_t norm_common(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma, float 
     return W8A8_OK;
 }
 
+// A host buffer: pinned or pageable host memory, not device or managed memory.
+w8a8_status_t check_host_ptr(const void *p)
+{
+    if (p == nullptr)
+        return W8A8_ERR_INVALID_ARG;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_INVALID_ARG;
+    }
+    return (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeUnregistered)
+               ? W8A8_OK
+               : W8A8_ERR_INVALID_ARG;
+}
+
+// Rows per chunk of w8a8_linear_host: the caller's, else 4 MiB of x per chunk rounded
+// down to 128 rows (at least 128); never more than M.
+int64_t host_chunk(int64_t M, int64_t K, int64_t chunk_rows)
+{
+    int64_t c = chunk_rows;
+    if (c <= 0) {
+        const int64_t per = K > 0 ? (int64_t{4} << 20) / (2 * K) : (int64_t{1} << 20);
+        c = std::max<int64_t>(128, per / 128 * 128);
+    }
+    return std::min(c, std::max<int64_t>(M, 1));
+}
+
+// The two copy streams and seven events of w8a8_linear_host, one set per device,
+// created by the first call on that device.
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_host_mu;      // one w8a8_linear_host enqueue at a time
+
+w8a8_status_t host_pipe(int dev, HostPipe *&hp)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    HostPipe &h = g_pipe[dev];
+    if (!h.ready) {
+        cudaError_t e = cudaStreamCreateWithFlags(&h.h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess)
+            e = cudaStreamCreateWithFlags(&h.d2h, cudaStreamNonBlocking);
+        cudaEvent_t *evs[7] = {&h.start, &h.h2d_done[0], &h.h2d_done[1], &h.comp_done[0],
+                               &h.comp_done[1], &h.d2h_done[0], &h.d2h_done[1]};
+        for (int i = 0; i < 7 && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(evs[i], cudaEventDisableTiming);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        h.ready = true;
+    }
+    hp = &h;
+    return W8A8_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -538,6 +596,136 @@ w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8
     W8A8_TRY(bf16_impl(x, w->w_bf16, bias, y, M, K, N, st));
     if (path_taken != nullptr)
         *path_taken = W8A8_PATH_BF16;
+    return W8A8_OK;
+}
+
+int64_t w8a8_linear_host_chunk_rows(int64_t M, int64_t K)
+{
+    return host_chunk(M, K, 0);
+}
+
+size_t w8a8_linear_host_workspace_bytes(int64_t M, int64_t K, int64_t N, int64_t chunk_rows)
+{
+    if (M <= 0 || K < 0 || N <= 0 || chunk_rows < 0)
+        return 0;
+    const int64_t C = host_chunk(M, K, chunk_rows);
+    return 2 * round256(static_cast<size_t>(C) * K * 2) + 2 * round256(static_cast<size_t>(C) * N * 2) +
+           w8a8_linear_workspace_bytes(C, K, N);
+}
+
+w8a8_status_t w8a8_linear_host(const w8a8_bf16_t *x_host, int64_t M, int64_t K,
+                               const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                               w8a8_bf16_t *y_host, void *workspace, size_t workspace_bytes,
+                               int64_t chunk_rows, int *path_taken, void *stream)
+{
+    if (path_taken != nullptr)
+        *path_taken = W8A8_PATH_NONE;
+    if (M < 0 || K < 0 || chunk_rows < 0 || chunk_rows % 128 != 0)
+        return W8A8_ERR_INVALID_ARG;
+    W8A8_TRY(check_weight(w, K));
+    const int64_t N = w->N;
+    if (M == 0 || N == 0)
+        return W8A8_OK;
+    if (K > 0)
+        W8A8_TRY(check_host_ptr(x_host));
+    W8A8_TRY(check_host_ptr(y_host));
+    if (K > 0)
+        W8A8_TRY(check_device_ptr(w->w_bf16));
+    if (bias != nullptr)
+        W8A8_TRY(check_device_ptr(bias));
+    const int64_t C = host_chunk(M, K, chunk_rows);
+    if (workspace == nullptr || !aligned16(workspace) ||
+        workspace_bytes < w8a8_linear_host_workspace_bytes(M, K, N, chunk_rows))
+        return W8A8_ERR_WORKSPACE;
+    W8A8_TRY(check_device_ptr(workspace));
+    // the guard of w8a8_linear, decided once for the whole input (the staging buffers are
+    // 256-byte aligned); every chunk then takes the same path
+    const bool int8 = int8_shape_ok(M, K, N) && w->wq != nullptr && aligned16(w->wq) &&
+                      (bias == nullptr || aligned16(bias));
+    if (int8) {
+        W8A8_TRY(check_device_ptr(w->wq));
+        W8A8_TRY(check_device_ptr(w->ws));
+    }
+    int dev;
+    W8A8_TRY(current_device(dev));
+    HostPipe *hp = nullptr;
+    W8A8_TRY(host_pipe(dev, hp));
+
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    const size_t xsz = round256(static_cast<size_t>(C) * K * 2);
+    const size_t ysz = round256(static_cast<size_t>(C) * N * 2);
+    uint16_t *xbuf[2] = {reinterpret_cast<uint16_t *>(base), reinterpret_cast<uint16_t *>(base + xsz)};
+    uint16_t *ybuf[2] = {reinterpret_cast<uint16_t *>(base + 2 * xsz),
+                         reinterpret_cast<uint16_t *>(base + 2 * xsz + ysz)};
+    int8_t *xq = reinterpret_cast<int8_t *>(base + 2 * xsz + 2 * ysz);
+    float *xs = reinterpret_cast<float *>(base + 2 * xsz + 2 * ysz + round256(static_cast<size_t>(C) * K));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t nch = (M + C - 1) / C;
+
+    std::lock_guard<std::mutex> lk(g_host_mu);
+    w8a8_status_t status = W8A8_OK;
+    cudaError_t e = cudaEventRecord(hp->start, st);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(hp->d2h, hp->start, 0);
+    int64_t done = 0;
+    for (int64_t i = 0; i < nch && e == cudaSuccess && status == W8A8_OK; ++i) {
+        const int b = static_cast<int>(i & 1);
+        const int64_t r0 = i * C, rows = std::min(C, M - r0);
+        // x chunk in: its buffer was last read by the linear on chunk i - 2
+        if (i >= 2)
+            e = cudaStreamWaitEvent(hp->h2d, hp->comp_done[b], 0);
+        if (e == cudaSuccess && K > 0)
+            e = cudaMemcpyAsync(xbuf[b], x_host + r0 * K, static_cast<size_t>(rows) * K * 2,
+                                cudaMemcpyHostToDevice, hp->h2d);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(hp->h2d_done[b], hp->h2d);
+        // the linear: after its x chunk landed and after chunk i - 2 left its y buffer
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(st, hp->h2d_done[b], 0);
+        if (e == cudaSuccess && i >= 2)
+            e = cudaStreamWaitEvent(st, hp->d2h_done[b], 0);
+        if (e != cudaSuccess)
+            break;
+        if (int8) {
+            status = quantize_impl(xbuf[b], rows, K, xq, xs, st);
+            if (status == W8A8_OK)
+                status = gemm_i8_impl(xq, xs, rows, K, w, bias, ybuf[b], st);
+        } else {
+            status = bf16_impl(xbuf[b], w->w_bf16, bias, ybuf[b], rows, K, N, st);
+        }
+        if (status != W8A8_OK)
+            break;
+        e = cudaEventRecord(hp->comp_done[b], st);
+        // y chunk out
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(hp->d2h, hp->comp_done[b], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(y_host + r0 * N, ybuf[b], static_cast<size_t>(rows) * N * 2,
+                                cudaMemcpyDeviceToHost, hp->d2h);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(hp->d2h_done[b], hp->d2h);
+        if (e == cudaSuccess)
+            done = i + 1;
+    }
+    // the caller's stream waits for the last copies back (both buffers), and for any copy
+    // in that an error left without its linear
+    if (e == cudaSuccess)
+        e = cudaEventRecord(hp->start, hp->h2d);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(st, hp->start, 0);
+    for (int64_t i = std::max<int64_t>(0, done - 2); i < done; ++i) {
+        const cudaError_t e2 = cudaStreamWaitEvent(st, hp->d2h_done[i & 1], 0);
+        if (e == cudaSuccess)
+            e = e2;
+    }
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    if (status != W8A8_OK)
+        return status;
+    if (path_taken != nullptr)
+        *path_taken = int8 ? W8A8_PATH_INT8 : W8A8_PATH_BF16;
     return W8A8_OK;
 }
 

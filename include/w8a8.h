@@ -157,6 +157,44 @@ W8A8_API w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, c
                           const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *workspace,
                           size_t workspace_bytes, int *path_taken, void *stream);
 
+/* Rows per chunk that w8a8_linear_host uses when chunk_rows is 0: 4 MiB of x per chunk
+ * (K BF16 values per row), rounded down to a multiple of 128 rows, at least 128. */
+W8A8_API int64_t w8a8_linear_host_chunk_rows(int64_t M, int64_t K);
+
+/* Bytes of device workspace w8a8_linear_host needs: two x chunks and two y chunks
+ * (C = the chunk rows in use: chunk_rows, or the default above, capped at M), each
+ * rounded up to 256 bytes, followed by w8a8_linear_workspace_bytes(C, K, N). */
+W8A8_API size_t w8a8_linear_host_workspace_bytes(int64_t M, int64_t K, int64_t N,
+                                                 int64_t chunk_rows);
+
+/* w8a8_linear on activations and outputs in HOST memory.  The operation and the guard
+ * are those of w8a8_linear (TurboT2VA paper, W8A8 operator and guard paragraphs); the
+ * streaming of host buffers through the GPU is this library's own.
+ *   x_host: [M, K] BF16 host buffer; y_host: [M, N] BF16 host buffer.  Pinned
+ *           (page-locked) memory lets the copies overlap; pageable memory works, slower.
+ *           Device or managed pointers here give W8A8_ERR_INVALID_ARG.
+ *   w, bias: as for w8a8_linear (device buffers).
+ *   workspace: device buffer of at least w8a8_linear_host_workspace_bytes(M, K, N,
+ *           chunk_rows) bytes, 16-byte aligned; else W8A8_ERR_WORKSPACE.
+ *   chunk_rows: rows per chunk, 0 for w8a8_linear_host_chunk_rows(M, K); a positive value
+ *           must be a multiple of 128 (else W8A8_ERR_INVALID_ARG).
+ * The guard is decided once for the whole [M, K] input exactly as w8a8_linear decides it
+ * (host pointers aside), and every chunk then takes that path, so y_host receives the
+ * same bits as w8a8_linear on device copies of x.  The rows go through the GPU in chunks:
+ * the copy of chunk i + 1 to the device, the linear on chunk i and the copy of chunk
+ * i - 1 back to y_host overlap on three streams.  The linear runs on `stream`; the copies
+ * run on two streams of the library's own, which the first call on each device creates
+ * (with seven events), so make that first call outside stream capture.  Everything is
+ * ordered after the work already enqueued on `stream`, and `stream` waits for the last
+ * copy back: when `stream` reaches the end of the call's work, y_host is complete.  Calls
+ * are enqueued one at a time (a lock per library); calls that share a workspace must be
+ * ordered on the same stream or synchronized. */
+W8A8_API w8a8_status_t w8a8_linear_host(const w8a8_bf16_t *x_host, int64_t M, int64_t K,
+                                        const w8a8_weight_t *w, const w8a8_bf16_t *bias,
+                                        w8a8_bf16_t *y_host, void *workspace,
+                                        size_t workspace_bytes, int64_t chunk_rows,
+                                        int *path_taken, void *stream);
+
 /* Largest M * K that w8a8_linear_noalloc accepts on the INT8 path (16 Mi elements,
  * e.g. M = K = 4096). */
 #define W8A8_NOALLOC_MAX_ELEMS (16777216LL)
