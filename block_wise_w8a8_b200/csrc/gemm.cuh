@@ -267,6 +267,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // When launched as a programmatic dependent of the activation quantizer, the set-up
+    // above overlaps the quantizer's last blocks; nothing below reads an operand or a
+    // scale before that grid has completed and its writes are visible.  A no-op otherwise.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp < EPI_WARP0) {
     regs_dec<kRegsControl>();
     if (warp == 0) {

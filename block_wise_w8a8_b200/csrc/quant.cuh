@@ -200,6 +200,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
         fence_barrier_init();
     }
     __syncthreads();
+    // A GEMM launched after this kernel as a programmatic dependent may start now: its CTAs
+    // take SMs as this kernel's CTAs leave them, set up, and wait (griddepcontrol.wait)
+    // for this grid's codes and scales before reading them.
+    asm volatile("griddepcontrol.launch_dependents;");
 
     if (warp == kQWarps) {
         // ------------------------------------------------------------ TMA producer

@@ -142,9 +142,11 @@ w8a8_status_t make_operand_map(CUtensorMap &m, const void *base, CUtensorMapData
                     CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// pdl: launch as a programmatic dependent of the kernel before it on the stream (the
+// activation quantizer), so the GEMM's set-up overlaps that kernel's tail.
 template <gemm::Mode kMode>
 w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
-                          cudaStream_t stream)
+                          cudaStream_t stream, bool pdl = false)
 {
     int dev;
     W8A8_TRY(current_device(dev));
@@ -195,6 +197,20 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
         }
     }
     const int grid = std::min(p.num_units, sms);
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(gemm::NUM_THREADS);
+        cfg.dynamicSmemBytes = gemm::kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+        return e == cudaSuccess ? launch_status() : cuda_fail(e);
+    }
     kern<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, stream>>>(ta, tb, p);
     return launch_status();
 }
@@ -265,7 +281,7 @@ w8a8_status_t check_weight(const w8a8_weight_t *w, int64_t K)
 w8a8_status_t gemm_i8_impl(const int8_t *xq, const float *xs, int64_t M, int64_t K,
                            const w8a8_weight_t *w, const uint16_t *bias, uint16_t *y,
                            cudaStream_t stream, const uint16_t *resid = nullptr,
-                           const uint16_t *gate = nullptr, int64_t gate_T = 1)
+                           const uint16_t *gate = nullptr, int64_t gate_T = 1, bool pdl = false)
 {
     gemm::Params p{};
     p.M = M;
@@ -279,8 +295,8 @@ w8a8_status_t gemm_i8_impl(const int8_t *xq, const float *xs, int64_t M, int64_t
     p.gate = gate;
     p.gate_T = gate_T;
     if (gate != nullptr)
-        return launch_gemm<gemm::Mode::kI8Gated>(xq, w->wq, p, stream);
-    return launch_gemm<gemm::Mode::kI8Scaled>(xq, w->wq, p, stream);
+        return launch_gemm<gemm::Mode::kI8Gated>(xq, w->wq, p, stream, pdl);
+    return launch_gemm<gemm::Mode::kI8Scaled>(xq, w->wq, p, stream, pdl);
 }
 
 w8a8_status_t bf16_impl(const uint16_t *x, const uint16_t *w, const uint16_t *bias, uint16_t *y,
@@ -588,7 +604,7 @@ w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8
         float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                               round256(static_cast<size_t>(M) * K));
         W8A8_TRY(quantize_impl(x, M, K, xq, xs, st));
-        W8A8_TRY(gemm_i8_impl(xq, xs, M, K, w, bias, y, st));
+        W8A8_TRY(gemm_i8_impl(xq, xs, M, K, w, bias, y, st, nullptr, nullptr, 1, true));
         if (path_taken != nullptr)
             *path_taken = W8A8_PATH_INT8;
         return W8A8_OK;
@@ -691,7 +707,7 @@ w8a8_status_t w8a8_linear_host(const w8a8_bf16_t *x_host, int64_t M, int64_t K,
         if (int8) {
             status = quantize_impl(xbuf[b], rows, K, xq, xs, st);
             if (status == W8A8_OK)
-                status = gemm_i8_impl(xq, xs, rows, K, w, bias, ybuf[b], st);
+                status = gemm_i8_impl(xq, xs, rows, K, w, bias, ybuf[b], st, nullptr, nullptr, 1, true);
         } else {
             status = bf16_impl(xbuf[b], w->w_bf16, bias, ybuf[b], rows, K, N, st);
         }
