@@ -60,6 +60,29 @@ def test_workspace_query_and_status_strings(lib):
     assert lib.w8a8_status_string(5).startswith(b"workspace")
 
 
+def test_host_linear_chunk_and_workspace_query(lib):
+    """w8a8_linear_host's size queries: 4 MiB of x per chunk in whole 128-row steps, at
+    least 128 rows, at most M; the workspace holds two x and two y chunks (each rounded up
+    to 256 bytes) and the quantizer's workspace for one chunk."""
+    lib.w8a8_linear_host_chunk_rows.restype = ctypes.c_int64
+    lib.w8a8_linear_host_chunk_rows.argtypes = [ctypes.c_int64] * 2
+    lib.w8a8_linear_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.w8a8_linear_host_workspace_bytes.argtypes = [ctypes.c_int64] * 4
+    lib.w8a8_linear_workspace_bytes.restype = ctypes.c_size_t
+    lib.w8a8_linear_workspace_bytes.argtypes = [ctypes.c_int64] * 3
+    assert lib.w8a8_linear_host_chunk_rows(4096, 4096) == 512
+    assert lib.w8a8_linear_host_chunk_rows(4096, 2048) == 1024
+    assert lib.w8a8_linear_host_chunk_rows(4096, 3000) == 640      # 699 rows, down to 640
+    assert lib.w8a8_linear_host_chunk_rows(4096, 65536) == 128     # at least 128
+    assert lib.w8a8_linear_host_chunk_rows(300, 4096) == 300       # at most M
+    r256 = lambda v: (v + 255) // 256 * 256
+    for M, K, N, c in [(4096, 4096, 4096, 0), (1024, 2048, 8192, 384), (1000, 256, 384, 256)]:
+        C = min(c or lib.w8a8_linear_host_chunk_rows(M, K), M)
+        want = 2 * r256(C * K * 2) + 2 * r256(C * N * 2) + lib.w8a8_linear_workspace_bytes(C, K, N)
+        assert lib.w8a8_linear_host_workspace_bytes(M, K, N, c) == want
+    assert lib.w8a8_linear_host_workspace_bytes(0, 4096, 4096, 0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     import block_wise_w8a8_b200 as w8
     monkeypatch.setattr(w8, "LIB_PATH", str(tmp_path / "missing.so"))
