@@ -5,10 +5,10 @@ C ABI, against the oracle.
 rstd must equal the oracle's bit for bit except on rows where the two FP64 sums, taken in
 different orders, round to neighbouring FP32 values (at most one ulp, on a vanishing
 fraction of rows); given the kernel's rstd, codes and scales must equal the oracle's bit
-for bit.  Shapes cover every cluster size (C = min(8, K / 128)), blocks resident between
-the passes (K / 128 / C <= 6) and reloaded, block counts per CTA that are not a multiple
-of the four consumer groups, CTAs with no block, gamma absent, and eps = 0 (the exact
-conversion path)."""
+for bit.  Shapes cover every cluster size (C = min(4, K / 128)), 1 to 128 blocks per CTA
+and strip, block counts per CTA that are not a multiple of the four consumer groups or
+differ between the CTAs of a cluster, more strips than clusters, gamma absent, and eps = 0
+(the exact conversion path)."""
 import numpy as np
 import pytest
 import torch
@@ -58,13 +58,14 @@ def _check(orc, x, g, eps, xq, xs, rstd, mod=None):
     np.testing.assert_array_equal(xq, q_ref)
 
 
-SHAPES = [(128, 128),      # C = 1
-          (256, 384),      # C = 3
-          (384, 896),      # C = 7, one block per CTA
-          (256, 6144),     # C = 8, six blocks per CTA: resident, the largest
-          (256, 7168),     # seven blocks per CTA: reloaded, not a multiple of 4
-          (128, 8192),     # eight blocks per CTA: reloaded
-          (1152, 2048)]    # more strips than one pass of clusters on small M
+SHAPES = [(128, 128),      # C = 1, one block
+          (256, 384),      # C = 3, one block per CTA
+          (384, 896),      # C = 4, seven blocks: 2, 2, 2, 1 per CTA
+          (256, 6144),     # 12 blocks per CTA
+          (256, 7168),     # 14 blocks per CTA: not a multiple of the 4 groups
+          (128, 8192),     # 16 blocks per CTA
+          (1152, 2048),    # nine strips, 4 blocks per CTA
+          (128, 65536)]    # 128 blocks per CTA: the longest rows tested
 
 
 @pytest.mark.parametrize("M,K", SHAPES)
