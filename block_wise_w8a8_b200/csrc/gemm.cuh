@@ -76,7 +76,7 @@ struct alignas(1024) Smem {
     uint64_t tempty[2];
     uint64_t mma_done;
     uint64_t sready[2];            // scale table sprod[b] written (all epilogue threads)
-    alignas(16) uint8_t stage[8][32 * 64];   // per epilogue warp: 32 rows x 64 bytes
+    alignas(1024) uint8_t stage[8][32 * 64]; // per epilogue warp: 32 rows x 64 bytes
     uint32_t tmem_base;
     int abort;
 };
@@ -86,7 +86,9 @@ static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA m
 // Byte offset of 16-byte piece c (0..3) of row r (0..31) in an epilogue warp's staging
 // buffer: rows of 64 bytes, pieces XOR-swizzled with (r / 2) % 4, so that a warp writing
 // one piece of each of its 32 rows, or reading 4 pieces of 8 rows, hits 32 distinct banks
-// in every quarter-warp phase.
+// in every quarter-warp phase.  This is the TMA's 64-byte swizzle (16-byte chunk index
+// XOR address bits 7-8) for a buffer aligned to 512 bytes, so a TMA store with
+// CU_TENSOR_MAP_SWIZZLE_64B reads the buffer back as plain rows.
 __device__ __forceinline__ uint32_t stage_off(int r, int c)
 {
     return static_cast<uint32_t>(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
@@ -172,6 +174,24 @@ __device__ __forceinline__ bool gemm_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// TMA store of one 2-D box from shared memory (bulk-group completion, no multicast), and
+// the waits on this thread's outstanding bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t c0,
+                                             int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the bulk stores issued by this thread have finished reading shared memory
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy writes to shared memory become visible to the TMA (async proxy)
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_l2(const void *p)
 {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -228,7 +248,7 @@ __device__ __forceinline__ void scales_fetch(float *sx, float (*sw)[KB_MAX], con
 template <Mode kMode>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Params p)
+                const __grid_constant__ CUtensorMap tmY, const Params p)
 {
     constexpr bool kInt8 = (kMode != Mode::kBf16);                    // INT8 operands
     constexpr bool kPerKb = (kMode == Mode::kI8Scaled || kMode == Mode::kI8Dump ||
@@ -258,6 +278,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_barrier_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        if (kMode == Mode::kI8Scaled)
+            prefetch_tensormap(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, TMEM_COLS);
@@ -507,7 +529,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int64_t m = static_cast<int64_t>(tm) * BM + row;
                 const int64_t n0 = static_cast<int64_t>(tn) * BN + hcol * 128;
                 const int64_t m_w = m - static_cast<int64_t>(lane);
-                if (active && n0 < p.N) {
+                if (kMode == Mode::kI8Scaled && active && n0 < p.N) {
+                    // Each round: the warp writes its 32 x 32 BF16 block into its staging
+                    // buffer and lane 0 hands it to the TMA, which stores it while the warp
+                    // goes on; the buffer is rewritten only after the TMA has read it.
+                    uint8_t *stg = sm.stage[ew];
+#pragma unroll
+                    for (int rd = 0; rd < 4; ++rd) {
+                        if (lane == 0)
+                            tma_store_wait_read();
+                        __syncwarp();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int c8 = rd * 4 + c;
+                            float bb[8];
+                            load_bias8(p.bias, n0 + c8 * 8, bb);
+                            uint32_t o[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                o[i] = pack_bf16x2(acc[c8 * 4 + i].x + bb[2 * i], acc[c8 * 4 + i].y + bb[2 * i + 1]);
+                            st_shared_v4(stg + stage_off(static_cast<int>(lane), c), make_uint4(o[0], o[1], o[2], o[3]));
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0)
+                            tma_store_2d(&tmY, stg, static_cast<int32_t>(n0 + rd * 32), static_cast<int32_t>(m_w));
+                    }
+                } else if (active && n0 < p.N) {
                     uint8_t *stg = sm.stage[ew];
                     const int pr = static_cast<int>(lane >> 2), pc = static_cast<int>(lane & 3);
                     const uint16_t *gp = kMode == Mode::kI8Gated ? p.gate + (m / p.gate_T) * p.N + n0 : nullptr;
@@ -561,6 +609,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
+            // the output stores still in flight complete before the CTA exits
+            if (kMode == Mode::kI8Scaled && lane == 0)
+                tma_store_wait_all();
         } else if (kMode == Mode::kI8Dump) {
             const int KB = static_cast<int>(p.K / 128);
             for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {

@@ -156,6 +156,12 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
     const int es = kInt8 ? 1 : 2;
     W8A8_TRY(make_operand_map(ta, a, dt, es, p0.M, p0.K, gemm::BM));
     W8A8_TRY(make_operand_map(tb, b, dt, es, p0.N, p0.K, gemm::BN));
+    // the block-scaled GEMM stores its output by TMA: 32 x 32 BF16 boxes (64-byte rows)
+    // from the epilogue warps' staging buffers, whose layout is the 64-byte swizzle
+    CUtensorMap ty = ta;
+    if (kMode == gemm::Mode::kI8Scaled)
+        W8A8_TRY(make_map(ty, p0.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p0.M, p0.N, 32, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B));
     gemm::Params p = p0;
     p.num_tm = static_cast<int32_t>((p.M + gemm::BM - 1) / gemm::BM);
     p.num_tn = static_cast<int32_t>((p.N + gemm::BN - 1) / gemm::BN);
@@ -208,10 +214,10 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
         attr.val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p);
         return e == cudaSuccess ? launch_status() : cuda_fail(e);
     }
-    kern<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, stream>>>(ta, tb, p);
+    kern<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, stream>>>(ta, tb, ty, p);
     return launch_status();
 }
 
