@@ -156,8 +156,8 @@ W8A8_API size_t w8a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N);
  * On the INT8 path two kernels run on `stream`: the activation quantizer, then the GEMM,
  * launched as a programmatic dependent of it (cudaLaunchAttributeProgrammaticStream-
  * Serialization): the GEMM's set-up overlaps the quantizer's last blocks and it reads
- * nothing before the quantizer has completed.  Stream order is unchanged for the caller,
- * and the pair can be captured into a CUDA graph like any two launches. */
+ * nothing before the quantizer has completed.  Stream order is unchanged for the
+ * caller. */
 W8A8_API w8a8_status_t w8a8_linear(const w8a8_bf16_t *x, int64_t M, int64_t K, const w8a8_weight_t *w,
                           const w8a8_bf16_t *bias, w8a8_bf16_t *y, void *workspace,
                           size_t workspace_bytes, int *path_taken, void *stream);
