@@ -89,3 +89,17 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(w8, "_lib", None)
     with pytest.raises(RuntimeError):
         w8.lib()
+
+
+def test_linear_host_binding_checks_its_input_first():
+    """The binding refuses a non-CPU x (a meta tensor stands in for a device tensor here)
+    and a non-BF16 x before it touches the weight or the library."""
+    import torch
+
+    import block_wise_w8a8_b200 as w8
+    with pytest.raises(ValueError):
+        w8.linear_host(torch.empty((128, 128), dtype=torch.bfloat16, device="meta"), None)
+    with pytest.raises(TypeError):
+        w8.linear_host(torch.zeros((128, 128), dtype=torch.float32), None)
+    with pytest.raises(TypeError):
+        w8.linear_host(torch.zeros((128, 256), dtype=torch.bfloat16)[:, ::2], None)
