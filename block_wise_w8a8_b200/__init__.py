@@ -129,13 +129,44 @@ def _need(t, dtype, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _out(t, shape, dtype, device, name):
+    """A caller-supplied output buffer: checked here, before the library writes into it,
+    for type, dtype, exact shape, device and contiguity (a wrong one would be written out
+    of bounds); None -> a new tensor."""
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=device)
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != torch.device(device):
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _in(t, shape, dtype, device, name):
+    """A required input buffer, checked like an output buffer."""
+    if t is None:
+        raise TypeError(f"{name} is required")
+    return _out(t, shape, dtype, device, name)
+
+
+def _block_scales(xs, M, K, device, name):
+    """A block-scale table [M/128, K/128] float32 on the device."""
+    return _out(xs, (M // 128, K // 128), torch.float32, device, name)
+
+
 def quantize_act(x, xq=None, xs=None):
     """Block-wise 128x128 INT8 quantization of a BF16 [M, K] matrix -> (xq int8 [M, K],
     xs float32 [M/128, K/128])."""
     _need(x, torch.bfloat16, "x")
     M, K = x.shape
-    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
-    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=x.device) if xs is None else xs
+    xq = _out(xq, (M, K), torch.int8, x.device, "xq")
+    xs = _block_scales(xs, M, K, x.device, "xs")
     _check("w8a8_quantize_act", lib().w8a8_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(xs),
                                                          _stream(x.device)))
     return xq, xs
@@ -158,8 +189,8 @@ def rowwise_quantize(x, q=None, s=None):
     For a weight [N, K] this gives its per-output-channel codes and scales."""
     _need(x, torch.bfloat16, "x")
     rows, K = x.shape
-    q = torch.empty((rows, K), dtype=torch.int8, device=x.device) if q is None else q
-    s = torch.empty((rows,), dtype=torch.float32, device=x.device) if s is None else s
+    q = _out(q, (rows, K), torch.int8, x.device, "q")
+    s = _out(s, (rows,), torch.float32, x.device, "s")
     _check("w8a8_rowwise_quantize", lib().w8a8_rowwise_quantize(_ptr(x), rows, K, _ptr(q), _ptr(s),
                                                                  _stream(x.device)))
     return q, s
@@ -171,9 +202,13 @@ def rowwise_linear_prequant(xq, xs, wq, ws, bias=None, out=None):
     _need(wq, torch.int8, "wq")
     M, K = xq.shape
     N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, {K}], got {tuple(wq.shape)}")
+    _in(xs, (M,), torch.float32, xq.device, "xs")
+    _in(ws, (N,), torch.float32, xq.device, "ws")
     if bias is not None:
-        _need(bias, torch.bfloat16, "bias")
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+        _out(bias, (N,), torch.bfloat16, xq.device, "bias")
+    y = _out(out, (M, N), torch.bfloat16, xq.device, "out")
     _check("w8a8_rowwise_linear", lib().w8a8_rowwise_linear(
         _ptr(xq), _ptr(xs), M, K, _ptr(wq), _ptr(ws), N, _ptr(bias), _ptr(y), _stream(xq.device)))
     return y
@@ -193,9 +228,11 @@ def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):
         _need(gamma, torch.bfloat16, "gamma")
     M, K = x.shape
     dev = x.device
-    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
-    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=dev) if xs is None else xs
-    rstd = torch.empty((M,), dtype=torch.float32, device=dev) if rstd is None else rstd
+    if gamma is not None:
+        _out(gamma, (K,), torch.bfloat16, dev, "gamma")
+    xq = _out(xq, (M, K), torch.int8, dev, "xq")
+    xs = _block_scales(xs, M, K, dev, "xs")
+    rstd = _out(rstd, (M,), torch.float32, dev, "rstd")
     _check("w8a8_rmsnorm_quantize_act",
            lib().w8a8_rmsnorm_quantize_act(_ptr(x), _ptr(gamma), float(eps), M, K, _ptr(xq),
                                            _ptr(xs), _ptr(rstd), _stream(dev)))
@@ -216,9 +253,11 @@ def rmsnorm_mod_quantize_act(x, gamma, scale, shift, eps=1e-6, xq=None, xs=None,
     if scale.shape != (B, K) or shift.shape != (B, K) or B == 0 or M % B:
         raise ValueError(f"scale and shift must be [B, {K}] with B dividing M = {M}")
     dev = x.device
-    xq = torch.empty((M, K), dtype=torch.int8, device=dev) if xq is None else xq
-    xs = torch.empty((M // 128, K // 128), dtype=torch.float32, device=dev) if xs is None else xs
-    rstd = torch.empty((M,), dtype=torch.float32, device=dev) if rstd is None else rstd
+    if gamma is not None:
+        _out(gamma, (K,), torch.bfloat16, dev, "gamma")
+    xq = _out(xq, (M, K), torch.int8, dev, "xq")
+    xs = _block_scales(xs, M, K, dev, "xs")
+    rstd = _out(rstd, (M,), torch.float32, dev, "rstd")
     _check("w8a8_rmsnorm_mod_quantize_act",
            lib().w8a8_rmsnorm_mod_quantize_act(_ptr(x), _ptr(gamma), _ptr(scale), _ptr(shift),
                                                M // B, float(eps), M, K, _ptr(xq), _ptr(xs),
@@ -236,6 +275,9 @@ class W8A8Weight:
         self.N, self.K = w_bf16.shape
         if wq is None and self.N % 128 == 0 and self.K % 128 == 0 and self.N and self.K:
             wq, ws = quantize_weight(w_bf16)
+        elif wq is not None:
+            _in(wq, (self.N, self.K), torch.int8, w_bf16.device, "wq")
+            _in(ws, (self.N // 128, self.K // 128), torch.float32, w_bf16.device, "ws")
         self.wq, self.ws = wq, ws
         self._rec = _Weight(self.N, self.K, w_bf16.data_ptr(),
                             0 if wq is None else wq.data_ptr(),
@@ -243,6 +285,16 @@ class W8A8Weight:
 
     def record(self):
         return ctypes.byref(self._rec)
+
+
+def _weight_on(weight, K, device):
+    """The weight matches the activations' K and lives on their device."""
+    if not isinstance(weight, W8A8Weight):
+        raise TypeError("weight must be a W8A8Weight")
+    if weight.K != K:
+        raise ValueError(f"weight has K = {weight.K}, the activations K = {K}")
+    if weight.w.device != torch.device(device):
+        raise ValueError(f"weight is on {weight.w.device}, the activations on {device}")
 
 
 def linear_workspace_bytes(M, K, N):
@@ -259,10 +311,15 @@ def linear(x, weight, bias=None, out=None, workspace=None, return_path=False):
     M = math.prod(x.shape[:-1])
     N = weight.N
     dev = x.device
-    out = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, device=dev) if out is None else out
+    _weight_on(weight, K, dev)
+    if bias is not None:
+        _out(bias, (N,), torch.bfloat16, dev, "bias")
+    out = _out(out, (*x.shape[:-1], N), torch.bfloat16, dev, "out")
     need = linear_workspace_bytes(M, K, N)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif workspace is not None:
+        _out(workspace, (workspace.numel(),), torch.uint8, dev, "workspace")
     path = ctypes.c_int(-1)
     _check("w8a8_linear", lib().w8a8_linear(
         _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
@@ -290,13 +347,19 @@ def linear_host(x, weight, bias=None, out=None, workspace=None, chunk_rows=0, re
     M = math.prod(x.shape[:-1])
     N = weight.N
     dev = weight.w.device
+    if weight.K != K:
+        raise ValueError(f"weight has K = {weight.K}, the activations K = {K}")
+    if bias is not None:
+        _out(bias, (N,), torch.bfloat16, dev, "bias")
     if out is None:
         out = torch.empty((*x.shape[:-1], N), dtype=torch.bfloat16, pin_memory=True)
-    elif out.device.type != "cpu" or out.dtype != torch.bfloat16 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous CPU torch.bfloat16 tensor")
+    else:
+        _out(out, (*x.shape[:-1], N), torch.bfloat16, "cpu", "out")
     need = linear_host_workspace_bytes(M, K, N, chunk_rows)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif workspace is not None:
+        _out(workspace, (workspace.numel(),), torch.uint8, dev, "workspace")
     path = ctypes.c_int(-1)
     _check("w8a8_linear_host", lib().w8a8_linear_host(
         _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), _ptr(workspace),
@@ -319,7 +382,10 @@ def linear_noalloc(x, weight, bias=None, out=None, return_path=False):
     K = x.shape[-1]
     M = math.prod(x.shape[:-1])
     dev = x.device
-    out = torch.empty((*x.shape[:-1], weight.N), dtype=torch.bfloat16, device=dev) if out is None else out
+    _weight_on(weight, K, dev)
+    if bias is not None:
+        _out(bias, (weight.N,), torch.bfloat16, dev, "bias")
+    out = _out(out, (*x.shape[:-1], weight.N), torch.bfloat16, dev, "out")
     path = ctypes.c_int(-1)
     _check("w8a8_linear_noalloc", lib().w8a8_linear_noalloc(
         _ptr(x), M, K, weight.record(), _ptr(bias), _ptr(out), ctypes.byref(path), _stream(dev)))
@@ -329,9 +395,12 @@ def linear_noalloc(x, weight, bias=None, out=None, return_path=False):
 def linear_prequant(xq, xs, weight, bias=None, out=None):
     """The INT8 block-scaled GEMM on already-quantized activations."""
     _need(xq, torch.int8, "xq")
-    _need(xs, torch.float32, "xs")
     M, K = xq.shape
-    out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _in(xs, (M // 128, K // 128), torch.float32, xq.device, "xs")
+    _weight_on(weight, K, xq.device)
+    if bias is not None:
+        _out(bias, (weight.N,), torch.bfloat16, xq.device, "bias")
+    out = _out(out, (M, weight.N), torch.bfloat16, xq.device, "out")
     _check("w8a8_linear_prequant", lib().w8a8_linear_prequant(
         _ptr(xq), _ptr(xs), M, K, weight.record(), _ptr(bias), _ptr(out), _stream(xq.device)))
     return out
@@ -342,14 +411,19 @@ def linear_prequant_gated(xq, xs, weight, resid, gate, bias=None, out=None):
     out = bf16(resid + gate[m // T] * (xq wq^T + bias)), T = M // gate.shape[0].  out may
     be resid itself (in-place update); by default a new tensor."""
     _need(xq, torch.int8, "xq")
-    _need(xs, torch.float32, "xs")
     _need(resid, torch.bfloat16, "resid")
     _need(gate, torch.bfloat16, "gate")
     M, K = xq.shape
+    _in(xs, (M // 128, K // 128), torch.float32, xq.device, "xs")
+    _weight_on(weight, K, xq.device)
     B = gate.shape[0]
     if resid.shape != (M, weight.N) or gate.shape != (B, weight.N) or B == 0 or M % B:
         raise ValueError(f"resid must be [{M}, {weight.N}] and gate [B, {weight.N}] with B dividing M")
-    out = torch.empty((M, weight.N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    if resid.device != xq.device or gate.device != xq.device:
+        raise ValueError("resid and gate must be on the device of xq")
+    if bias is not None:
+        _out(bias, (weight.N,), torch.bfloat16, xq.device, "bias")
+    out = _out(out, (M, weight.N), torch.bfloat16, xq.device, "out")
     _check("w8a8_linear_prequant_gated", lib().w8a8_linear_prequant_gated(
         _ptr(xq), _ptr(xs), M, K, weight.record(), _ptr(bias), _ptr(resid), _ptr(gate), M // B,
         _ptr(out), _stream(xq.device)))
@@ -362,7 +436,11 @@ def bf16_linear(x, w, bias=None, out=None):
     _need(w, torch.bfloat16, "w")
     M, K = x.shape
     N = w.shape[0]
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    if w.shape[1] != K or w.device != x.device:
+        raise ValueError(f"w must be [N, {K}] on {x.device}")
+    if bias is not None:
+        _out(bias, (N,), torch.bfloat16, x.device, "bias")
+    out = _out(out, (M, N), torch.bfloat16, x.device, "out")
     _check("w8a8_bf16_linear", lib().w8a8_bf16_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(out),
                                                        M, K, N, _stream(x.device)))
     return out

@@ -29,3 +29,15 @@ def assert_close_bf16(y_gpu_bits, ref_f32, orc, what=""):
     assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
                            f"worst err {float(err.max())} at {np.unravel_index(np.argmax(err - lim), err.shape)}")
     return float(err.max()), float((err / (np.abs(ref_b) + 1e-30)).max())
+
+
+def assert_codes_equal(q_gpu, s_gpu, q_ref, s_ref, what=""):
+    """GPU codes (int8) and scales (float32) against the oracle's own, bit for bit."""
+    q = q_gpu.detach().cpu().numpy() if isinstance(q_gpu, torch.Tensor) else np.asarray(q_gpu)
+    s = s_gpu.detach().cpu().numpy() if isinstance(s_gpu, torch.Tensor) else np.asarray(s_gpu)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    s_ref = np.ascontiguousarray(s_ref, dtype=np.float32)
+    bad_s = s.view(np.uint32) != s_ref.view(np.uint32)
+    assert not bad_s.any(), f"{what}: {int(bad_s.sum())} scales differ, first at {np.argwhere(bad_s)[0]}"
+    bad_q = q != q_ref
+    assert not bad_q.any(), f"{what}: {int(bad_q.sum())} codes differ, first at {np.argwhere(bad_q)[0]}"

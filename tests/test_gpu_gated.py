@@ -2,16 +2,18 @@
 paper, fused-operator paragraph), on the GPU through the C ABI, against the oracle:
 out = bf16(fl(r + fl(gate[m / T, n] * v))) with v the FP32 linear output.
 
-The block-wise GEMM's FP32 sums are compared with the tolerance of the linear layer
-(1e-2 + 1e-2 |ref|); the gate and residual arithmetic itself is checked exactly through
-special cases (gate 0 gives the residual, gate 1 on a zero residual gives the plain
-linear's bits) and in-place use (out aliasing the residual)."""
+The oracle quantizes x and w itself and runs the linear and the gated update on its own
+codes; the GPU's codes and scales must equal the oracle's bit for bit (so both sides
+multiply the same integers), and the outputs are compared with the tolerance of the
+linear layer (1e-2 + 1e-2 |ref|).  The gate and residual arithmetic itself is checked
+exactly through special cases (gate 0 gives the residual, gate 1 on a zero residual gives
+the plain linear's bits) and in-place use (out aliasing the residual)."""
 import numpy as np
 import pytest
 import torch
 
 import block_wise_w8a8_b200 as w8
-from gpu_util import assert_close_bf16, bf16_to_f32, dev_bf16, host_bits
+from gpu_util import assert_close_bf16, assert_codes_equal, bf16_to_f32, dev_bf16, host_bits
 from synth import f64_to_bf16_bits, workload
 
 pytestmark = pytest.mark.gpu
@@ -44,8 +46,11 @@ def test_gated_small(orc, M, K, N, T, with_bias):
     xq, xs = w8.quantize_act(dev_bf16(x))
     out = w8.linear_prequant_gated(xq, xs, wt, dev_bf16(res), dev_bf16(g),
                                    None if b is None else dev_bf16(b))
-    v = orc.w8a8_linear(xq.cpu().numpy(), xs.cpu().numpy(), wt.wq.cpu().numpy(),
-                        wt.ws.cpu().numpy(), b)
+    xq_ref, xs_ref = orc.block_quantize(x)
+    wq_ref, ws_ref = orc.block_quantize(w)
+    assert_codes_equal(xq, xs, xq_ref, xs_ref, "x")
+    assert_codes_equal(wt.wq, wt.ws, wq_ref, ws_ref, "w")
+    v = orc.w8a8_linear(xq_ref, xs_ref, wq_ref, ws_ref, b)
     ref = orc.gated_residual(v, res, g, T, M)
     assert_close_bf16(host_bits(out), bf16_to_f32(ref), orc, f"gated {M}x{K}x{N} T={T}")
     # in place: the residual buffer itself receives the update, same bits
@@ -85,12 +90,23 @@ def test_gated_hires_out_projection_sampled(orc):
     wt = w8.W8A8Weight(dev_bf16(w))
     xq, xs = w8.quantize_act(dev_bf16(x))
     out = host_bits(w8.linear_prequant_gated(xq, xs, wt, dev_bf16(res), dev_bf16(g)))
+    # all 32768 x 4096 activation codes and the whole weight, against the oracle's own
+    xq_ref, xs_ref = orc.block_quantize(x)
+    wq_ref, ws_ref = orc.block_quantize(w)
+    assert_codes_equal(xq, xs, xq_ref, xs_ref, "x")
+    assert_codes_equal(wt.wq, wt.ws, wq_ref, ws_ref, "w")
     r = np.random.default_rng(11)
     ms, ns = r.integers(0, M, 4096), r.integers(0, N, 4096)
-    v = orc.w8a8_linear_at(xq.cpu().numpy(), xs.cpu().numpy(), wt.wq.cpu().numpy(),
-                           wt.ws.cpu().numpy(), None, ms, ns)
+    v = orc.w8a8_linear_at(xq_ref, xs_ref, wq_ref, ws_ref, None, ms, ns)
     ref = orc.gated_residual(v, res[ms, ns], g, M, M, ms, ns)
-    assert_close_bf16(out[ms, ns], bf16_to_f32(ref), orc, "gated out projection")
+    assert_close_bf16(out[ms, ns], bf16_to_f32(ref), orc, "gated out projection (sampled)")
+    # and one whole 128-row strip
+    rows = slice(128 * 200, 128 * 201)
+    v = orc.w8a8_linear(xq_ref, xs_ref, wq_ref, ws_ref, None, m0=128 * 200, rows=128)
+    ref = orc.gated_residual(v, res[rows], g, M, M, np.repeat(np.arange(128 * 200, 128 * 201), N),
+                             np.tile(np.arange(N), 128))
+    assert_close_bf16(out[rows].reshape(-1), bf16_to_f32(ref).reshape(-1), orc,
+                      "gated out projection (strip 200)")
 
 
 def test_gated_errors():

@@ -157,3 +157,34 @@ def test_mod_errors():
     assert f(P(x), None, P(m), P(m), 128, -1.0, 256, 256, P(q), P(s), None, st) == 1
     assert L.w8a8_rmsnorm_quantize_act(P(x), None, 1e-6, 256, 200, P(q), P(s), None, st) == 2
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("modulated", [False, True])
+@pytest.mark.parametrize("eps", [0.0, 1e-6])
+def test_fused_codes_near_ties_exhaustive(orc, modulated, eps):
+    """Every BF16 value of both signs in [A/512, A] as a normalised value, for five block
+    absmaxes A that are not powers of two: the rows' RMS is 1 (rstd exactly 1.0), so the
+    fused kernel quantizes the input values themselves, and its codes and scales must
+    equal the oracle's bit for bit, near-ties included (eps = 0 takes the exact-square
+    instantiation, eps = 1e-6 the scaled one; modulated with zero scale and shift)."""
+    from norm_sweep import ABSMAXES, unit_rms_rows
+    K = 4096
+    x = unit_rms_rows(K, eps)
+    M = x.shape[0]
+    if modulated:
+        z = np.zeros((1, K), dtype=np.uint16)
+        xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), None, dev_bf16(z), dev_bf16(z), eps)
+    else:
+        xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), None, eps)
+    rstd = rstd.cpu().numpy()
+    assert np.all(rstd == 1.0)
+    xq, xs = xq.cpu().numpy(), xs.cpu().numpy()
+    q_ref, s_ref = orc.block_quantize(x)            # rstd = 1: the normalised values are x
+    np.testing.assert_array_equal(xs.view(np.uint32), s_ref.view(np.uint32))
+    for i, A in enumerate(ABSMAXES):
+        assert xs[i, 0] == np.float32(np.float32(A) / np.float32(127.0))
+    np.testing.assert_array_equal(xq, q_ref)
+    if modulated:
+        _check(orc, x, None, eps, xq, xs, rstd, (z, z, M))
+    else:
+        _check(orc, x, None, eps, xq, xs, rstd)

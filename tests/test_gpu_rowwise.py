@@ -1,17 +1,18 @@
 """The per-row / per-output-channel post-scale W8A8 operator (TurboT2VA paper, W8A8
 operator paragraph) on the GPU, through the C ABI, against the oracle.
 
-Codes and scales must be bit-exact.  The kernel's epilogue performs the oracle's FP32
-operations in the oracle's order (the INT32 sum rounded to FP32, the scale product, the
-product, the bias, one rounding each, no fused multiply-add), so its BF16 outputs must
-equal the oracle's FP32 outputs rounded to BF16 bit for bit; the tolerance bar of the
-block-wise path (1e-2 + 1e-2 |ref|) is checked as well."""
+Codes and scales must be bit-exact.  The oracle quantizes x and w itself and its linear
+runs on its own codes.  The kernel's epilogue performs the oracle's FP32 operations in
+the oracle's order (the INT32 sum rounded to FP32, the scale product, the product, the
+bias, one rounding each, no fused multiply-add), so its BF16 outputs must equal the
+oracle's FP32 outputs rounded to BF16 bit for bit; the tolerance bar of the block-wise
+path (1e-2 + 1e-2 |ref|) is checked as well."""
 import numpy as np
 import pytest
 import torch
 
 import block_wise_w8a8_b200 as w8
-from gpu_util import assert_close_bf16, dev_bf16, host_bits
+from gpu_util import assert_close_bf16, assert_codes_equal, dev_bf16, host_bits
 from synth import f64_to_bf16_bits, workload
 
 pytestmark = pytest.mark.gpu
@@ -50,7 +51,11 @@ def _check_linear(orc, x, w, b, what):
     xq, xs = w8.rowwise_quantize(dev_bf16(x))
     wq, ws = w8.rowwise_quantize(dev_bf16(w))
     y = w8.rowwise_linear_prequant(xq, xs, wq, ws, None if b is None else dev_bf16(b))
-    ref = orc.row_linear(xq.cpu().numpy(), xs.cpu().numpy(), wq.cpu().numpy(), ws.cpu().numpy(), b)
+    xq_ref, xs_ref = orc.row_quantize(x)
+    wq_ref, ws_ref = orc.row_quantize(w)
+    assert_codes_equal(xq, xs, xq_ref, xs_ref, f"{what} x")
+    assert_codes_equal(wq, ws, wq_ref, ws_ref, f"{what} w")
+    ref = orc.row_linear(xq_ref, xs_ref, wq_ref, ws_ref, b)
     yb = host_bits(y)
     np.testing.assert_array_equal(yb, orc.f32_to_bf16(ref), err_msg=what)
     assert_close_bf16(yb, ref, orc, what)
@@ -83,25 +88,26 @@ def test_rowwise_int32_sum_rounding(orc):
 
 
 def test_rowwise_linear_attn_proj_4096(orc):
-    """The 4096^3 workload: codes and scales of a 256-row slice and of all weight rows,
-    outputs at 4096 sampled points against the oracle."""
+    """The 4096^3 workload: codes and scales of all 4096 activation rows and all weight
+    rows, outputs on a 128-row strip and at 4096 sampled points, against the oracle on its
+    own codes."""
     wl = workload("attn_proj_4096")
     lin = wl.linears[0]
     xb = wl.x(4096, 4096)
     wb = wl.w(lin)
     xq, xs = w8.rowwise_quantize(dev_bf16(xb))
     wq, ws = w8.rowwise_quantize(dev_bf16(wb))
-    q_ref, s_ref = orc.row_quantize(xb[:256])
-    np.testing.assert_array_equal(xq[:256].cpu().numpy(), q_ref)
-    np.testing.assert_array_equal(xs[:256].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    q_ref, s_ref = orc.row_quantize(xb)
+    assert_codes_equal(xq, xs, q_ref, s_ref, "x")
     wq_ref, ws_ref = orc.row_quantize(wb)
-    np.testing.assert_array_equal(wq.cpu().numpy(), wq_ref)
-    np.testing.assert_array_equal(ws.cpu().numpy().view(np.uint32), ws_ref.view(np.uint32))
+    assert_codes_equal(wq, ws, wq_ref, ws_ref, "w")
     y = host_bits(w8.rowwise_linear_prequant(xq, xs, wq, ws))
     r = np.random.default_rng(7)
     ms, ns = r.integers(0, 4096, 4096), r.integers(0, 4096, 4096)
-    ref = orc.row_linear_at(xq.cpu().numpy(), xs.cpu().numpy(), wq_ref, ws_ref, None, ms, ns)
+    ref = orc.row_linear_at(q_ref, s_ref, wq_ref, ws_ref, None, ms, ns)
     np.testing.assert_array_equal(y[ms, ns], orc.f32_to_bf16(ref))
+    ref = orc.row_linear(q_ref, s_ref, wq_ref, ws_ref, None, m0=1920, rows=128)
+    np.testing.assert_array_equal(y[1920:2048], orc.f32_to_bf16(ref))
 
 
 def test_rowwise_errors():
