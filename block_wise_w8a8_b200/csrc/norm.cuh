@@ -11,8 +11,9 @@
 // and y is block-quantized exactly as quant.cuh does (scale max|y| / 127, codes
 // rne(fl32(y / s)) clamped to +-127), without being written out.
 //
-// Work split.  A cluster of C <= 8 CTAs owns one 128-row strip at a time; CTA r handles
-// the strip's 128-column blocks kb = r, r + C, ...  (nb of them).  Each CTA streams its
+// Work split.  A cluster of C = min(kMaxCluster, K / 128) CTAs (kMaxCluster = 4) owns one
+// 128-row strip at a time; CTA r handles the strip's 128-column blocks kb = r, r + C, ...
+// (nb of them).  Each CTA streams its
 // blocks into a ring of six 32 KB shared-memory slots with 2-D TMA loads (two 64-column
 // boxes per block, 128-byte swizzle, no multicast), each block twice: once for the sums of
 // squares and once for the codes.  The second load comes about one strip later and is

@@ -371,8 +371,9 @@ w8a8_status_t noalloc_scratch(int dev, void *&ptr)
     return W8A8_OK;
 }
 
-// Fused RMSNorm (+ modulation) + block quantization: clusters of C = min(8, K / 128) CTAs,
-// one cluster per 128-row strip at a time, as many clusters as fit on the device.
+// Fused RMSNorm (+ modulation) + block quantization: clusters of C = min(4, K / 128) CTAs
+// (4 = norm::kMaxCluster), one cluster per 128-row strip at a time, as many clusters as
+// fit on the device.
 template <bool kMod, bool kExactSq>
 w8a8_status_t launch_norm(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
 {
