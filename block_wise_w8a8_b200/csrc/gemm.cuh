@@ -70,6 +70,10 @@ struct alignas(1024) Smem {
     uint8_t b[STAGES][B_BYTES];
     float sx[2][KB_MAX];           // [tile parity][kb]: xs[tm, kb]
     float sw[2][2][KB_MAX];        // [tile parity][N half][kb]: ws[2 tn + half, kb]
+    // [tile % 3][column]: bias[256 tn + c] (BF16).  Three copies: the copy for tile i + 1
+    // is fetched at the start of tile i, while a slower warp may still be storing tile
+    // i - 1 (sx and sw, read only inside the K loop, need two).
+    alignas(16) uint16_t sbias[3][BN];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t tfull[2];
@@ -197,20 +201,14 @@ __device__ __forceinline__ void prefetch_l2(const void *p)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// Eight BF16 bias values (or zeros) as FP32.
-__device__ __forceinline__ void load_bias8(const uint16_t *bias, int64_t n, float (&bb)[8])
+// Eight BF16 bias values from the tile's copy in shared memory, as FP32.
+__device__ __forceinline__ void load_bias8_smem(const uint16_t *b, float (&bb)[8])
 {
-    if (bias != nullptr) {
-        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(bias + n));
-        bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
-        bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
-        bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
-        bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            bb[i] = 0.0f;
-    }
+    const uint4 bv = ld_shared_v4(b);
+    bb[0] = bf16_lo(bv.x); bb[1] = bf16_hi(bv.x);
+    bb[2] = bf16_lo(bv.y); bb[3] = bf16_hi(bv.y);
+    bb[4] = bf16_lo(bv.z); bb[5] = bf16_hi(bv.z);
+    bb[6] = bf16_lo(bv.w); bb[7] = bf16_hi(bv.w);
 }
 
 // The block scales a tile needs, copied global -> shared with cp.async by the epilogue
@@ -221,16 +219,30 @@ __device__ __forceinline__ void cp_async_4(void *dst, const void *src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-__device__ __forceinline__ void scales_fetch(float *sx, float (*sw)[KB_MAX], const Params &p,
-                                             int tm, int tn, int etid, int nthreads)
+// The tile's bias columns go to sbias the same way (16 bytes a thread, zeros past N or
+// without a bias), so that the tile's final phase reads them from shared memory.
+__device__ __forceinline__ void scales_fetch(float *sx, float (*sw)[KB_MAX], uint16_t *sbias,
+                                             const Params &p, int tm, int tn, int etid, int nthreads)
 {
     const int KB = static_cast<int>(p.K / 128);
     const int NB = static_cast<int>(p.N / 128);
+    if (etid < BN / 8) {
+        const int64_t n = static_cast<int64_t>(tn) * BN + etid * 8;
+        if (p.bias != nullptr && n < p.N)
+            cp_async_16(sbias + etid * 8, p.bias + n);
+        else
+            *reinterpret_cast<uint4 *>(sbias + etid * 8) = make_uint4(0, 0, 0, 0);
+    }
     for (int i = etid; i < 3 * KB; i += nthreads) {
         const int which = i / KB, kb = i - which * KB;
         if (which == 0) {
@@ -428,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (static_cast<int>(blockIdx.x) < p.num_units) {
                 int tm, tn, hs;
                 unit_coords(blockIdx.x, p, tm, tn, hs);
-                scales_fetch(sm.sx[0], sm.sw[0], p, tm, tn, etid, kEpiThreads);
+                scales_fetch(sm.sx[0], sm.sw[0], sm.sbias[0], p, tm, tn, etid, kEpiThreads);
                 cp_async_wait_all();
             }
             mbar_arrive(&sm.sready[0]);
@@ -452,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (tnext < p.num_units) {
                     int tm2, tn2, hs2;
                     unit_coords(tnext, p, tm2, tn2, hs2);
-                    scales_fetch(sm.sx[sb ^ 1], sm.sw[sb ^ 1], p, tm2, tn2, etid, kEpiThreads);
+                    scales_fetch(sm.sx[sb ^ 1], sm.sw[sb ^ 1], sm.sbias[(tile_iter + 1) % 3], p, tm2, tn2, etid, kEpiThreads);
                 }
                 if (kMode == Mode::kI8Gated && active) {
                     const int64_t pm = static_cast<int64_t>(tm) * BM + row;
@@ -543,7 +555,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int c = 0; c < 4; ++c) {
                             const int c8 = rd * 4 + c;
                             float bb[8];
-                            load_bias8(p.bias, n0 + c8 * 8, bb);
+                            load_bias8_smem(sm.sbias[tile_iter % 3] + hcol * 128 + c8 * 8, bb);
                             uint32_t o[4];
 #pragma unroll
                             for (int i = 0; i < 4; ++i)
@@ -577,7 +589,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int c = 0; c < 4; ++c) {
                             const int c8 = rd * 4 + c;
                             float bb[8];
-                            load_bias8(p.bias, n0 + c8 * 8, bb);
+                            load_bias8_smem(sm.sbias[tile_iter % 3] + hcol * 128 + c8 * 8, bb);
                             uint32_t o[4];
                             if (kMode == Mode::kI8Gated) {
                                 // gated residual update (TurboT2VA paper, fused-operator

@@ -61,10 +61,13 @@ def _check(orc, x, g, eps, xq, xs, rstd, mod=None):
 SHAPES = [(128, 128),      # C = 1, one block
           (256, 384),      # C = 3, one block per CTA
           (384, 896),      # C = 4, seven blocks: 2, 2, 2, 1 per CTA
+          (1152, 2048),    # nine strips, 4 blocks per CTA
+          (256, 2560),     # 20 blocks: 5 per CTA, not a multiple of the 4 groups
+          (384, 3968),     # 31 blocks: 8, 8, 8, 7 per CTA
+          (2304, 4096),    # 18 strips of the chain's row length, 8 blocks per CTA
           (256, 6144),     # 12 blocks per CTA
           (256, 7168),     # 14 blocks per CTA: not a multiple of the 4 groups
           (128, 8192),     # 16 blocks per CTA
-          (1152, 2048),    # nine strips, 4 blocks per CTA
           (128, 65536)]    # 128 blocks per CTA: the longest rows tested
 
 
@@ -78,7 +81,8 @@ def test_rmsnorm_quantize(orc, M, K, with_gamma):
 
 
 @pytest.mark.parametrize("M,K,T", [(256, 384, 128), (384, 896, 384), (512, 6144, 256),
-                                   (256, 7168, 128), (640, 1024, 128)])
+                                   (256, 7168, 128), (640, 1024, 128), (1024, 2560, 256),
+                                   (2304, 4096, 768)])
 @pytest.mark.parametrize("with_gamma", [True, False])
 def test_mod_rmsnorm_quantize(orc, M, K, T, with_gamma):
     r = np.random.default_rng(M + K + T)
@@ -188,3 +192,4 @@ def test_fused_codes_near_ties_exhaustive(orc, modulated, eps):
         _check(orc, x, None, eps, xq, xs, rstd, (z, z, M))
     else:
         _check(orc, x, None, eps, xq, xs, rstd)
+
