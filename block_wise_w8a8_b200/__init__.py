@@ -64,6 +64,7 @@ _SIGS = {
     "w8a8_bf16_linear": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                          ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p],
     "w8a8_debug_block_sums": [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                               ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p],
     "w8a8_debug_wait_timeout": [ctypes.c_uint64, ctypes.c_void_p],
     "w8a8_rowwise_quantize": [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
@@ -446,15 +447,21 @@ def bf16_linear(x, w, bias=None, out=None):
     return out
 
 
-def debug_block_sums(xq, wq):
-    """INT32 per-K-block partial products [M, N, K/128] from the tensor-core main loop."""
+def debug_block_sums(xq, wq, m0=0, rows=None, n0=0, cols=None):
+    """INT32 per-K-block partial products [rows, cols, K/128] of the window rows m0 ..
+    m0 + rows - 1, columns n0 .. n0 + cols - 1 (default: everything), from the tensor-core
+    main loop."""
     _need(xq, torch.int8, "xq")
     _need(wq, torch.int8, "wq")
     M, K = xq.shape
     N = wq.shape[0]
-    out = torch.empty((M, N, K // 128), dtype=torch.int32, device=xq.device)
+    if wq.shape[1] != K or wq.device != xq.device:
+        raise ValueError(f"wq must be [N, {K}] on {xq.device}")
+    rows = M - m0 if rows is None else rows
+    cols = N - n0 if cols is None else cols
+    out = torch.empty((rows, cols, K // 128), dtype=torch.int32, device=xq.device)
     _check("w8a8_debug_block_sums", lib().w8a8_debug_block_sums(
-        _ptr(xq), _ptr(wq), M, K, N, _ptr(out), _stream(xq.device)))
+        _ptr(xq), _ptr(wq), M, K, N, m0, rows, n0, cols, _ptr(out), _stream(xq.device)))
     return out
 
 

@@ -10,7 +10,7 @@
 //               running sums held in registers.  After the last block: + bias, BF16 store.
 //   kI8Gated  : kI8Scaled with the gated residual update of the TurboT2VA paper's fused-
 //               operator paragraph in the epilogue: y = bf16(r + gate[m / T] * v).
-//   kI8Dump   : same main loop; the epilogue writes P[m,n,kb] itself (test hook).
+//   kI8Dump   : same main loop; the epilogue writes P[m,n,kb] of a window itself (test hook).
 //   kBf16     : BF16 x BF16 -> FP32 GEMM (kind::f16) for the guard's fallback (TurboT2VA
 //               paper, guard paragraph), FP32 accumulation over all of K in tensor memory.
 //   kI8Row    : the per-row / per-output-channel post-scale W8A8 operator (TurboT2VA
@@ -114,7 +114,11 @@ struct Params {
     const uint16_t *resid;    // [M, N] BF16
     const uint16_t *gate;     // [M / gate_T, N] BF16
     int64_t gate_T;
-    int32_t *dump;            // [M, N, K/128] (dump mode)
+    // dump mode: P[m, n, kb] of the window rows dm0 .. dm0 + drows - 1, columns
+    // dn0 .. dn0 + dcols - 1 (relative to this launch's operands) into dump, laid out
+    // [drows, dcols, K/128]
+    int32_t *dump;
+    int64_t dm0, drows, dn0, dcols;
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_tm, int num_tn, int &tm, int &tn)
@@ -645,11 +649,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         uint32_t r[32];
                         tmem_ld32(tb + c * 32, r);
                         tmem_wait_ld();
-                        if (n0 < p.N) {
+                        const int64_t wm = m - p.dm0;
+                        if (n0 < p.N && wm >= 0 && wm < p.drows) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j) {
                                 const float v = __uint_as_float(r[j]) - kAccInitF;
-                                p.dump[(m * p.N + n0 + c * 32 + j) * KB + kb] = static_cast<int32_t>(v);
+                                const int64_t wn = n0 + c * 32 + j - p.dn0;
+                                if (wn >= 0 && wn < p.dcols)
+                                    p.dump[(wm * p.dcols + wn) * KB + kb] = static_cast<int32_t>(v);
                             }
                         }
                         tmem_st16(tb + c * 32, fill);

@@ -923,23 +923,35 @@ w8a8_status_t w8a8_rowwise_linear(const int8_t *xq, const float *xs, int64_t M, 
 }
 
 w8a8_status_t w8a8_debug_block_sums(const int8_t *xq, const int8_t *wq, int64_t M, int64_t K,
-                                    int64_t N, int32_t *out, void *stream)
+                                    int64_t N, int64_t m0, int64_t rows, int64_t n0, int64_t cols,
+                                    int32_t *out, void *stream)
 {
-    if (M < 0 || K < 0 || N < 0)
+    if (M < 0 || K < 0 || N < 0 || m0 < 0 || rows < 0 || n0 < 0 || cols < 0 || m0 + rows > M ||
+        n0 + cols > N)
         return W8A8_ERR_INVALID_ARG;
     if (!int8_shape_ok(M, K, N))
         return W8A8_ERR_SHAPE;
+    if (rows == 0 || cols == 0)
+        return W8A8_OK;
     W8A8_TRY(check_device_ptr(xq));
     W8A8_TRY(check_device_ptr(wq));
     W8A8_TRY(check_device_ptr(out));
     if (!aligned16(xq) || !aligned16(wq))
         return W8A8_ERR_ALIGNMENT;
+    // the main loop runs over the 128-aligned rows and columns that cover the window only
+    const int64_t mb0 = m0 / 128, mb1 = (m0 + rows + 127) / 128;
+    const int64_t nb0 = n0 / 128, nb1 = (n0 + cols + 127) / 128;
     gemm::Params p{};
-    p.M = M;
-    p.N = N;
+    p.M = (mb1 - mb0) * 128;
+    p.N = (nb1 - nb0) * 128;
     p.K = K;
     p.dump = out;
-    return launch_gemm<gemm::Mode::kI8Dump>(xq, wq, p, static_cast<cudaStream_t>(stream));
+    p.dm0 = m0 - mb0 * 128;
+    p.drows = rows;
+    p.dn0 = n0 - nb0 * 128;
+    p.dcols = cols;
+    return launch_gemm<gemm::Mode::kI8Dump>(xq + mb0 * 128 * K, wq + nb0 * 128 * K, p,
+                                            static_cast<cudaStream_t>(stream));
 }
 
 int w8a8_device_error(void)

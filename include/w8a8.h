@@ -292,11 +292,18 @@ W8A8_API w8a8_status_t w8a8_rowwise_linear(const int8_t *xq, const float *xs, in
                                            const w8a8_bf16_t *bias, w8a8_bf16_t *y,
                                            void *stream);
 
-/* Test hook: the INT32 partial products P[m, n, kb] of the INT8 GEMM, written by the
- * same tensor-core main loop as w8a8_linear, for xq [M, K] and wq [N, K] (M, K, N
- * multiples of 128).  out: [M, N, K/128] INT32 device buffer. */
+/* Test hook: the INT32 partial products P[m, n, kb] = sum over the 128 k of K block kb of
+ * xq[m, k] wq[n, k] (TurboT2VA paper, W8A8 operator paragraph: INT32 accumulation; the
+ * block-wise strategy's per-K-block sums), written by the same tensor-core main loop as
+ * w8a8_linear, for xq [M, K] and wq [N, K] (M, K, N multiples of 128, else
+ * W8A8_ERR_SHAPE) on the window of rows m0 .. m0 + rows - 1 and columns n0 .. n0 + cols -
+ * 1 (any offsets and sizes inside [M, N], else W8A8_ERR_INVALID_ARG).  out: [rows, cols,
+ * K/128] INT32 device buffer, caller-owned.  The main loop covers only the 128-aligned
+ * rows and columns around the window, so full-size operands can be spot-checked.
+ * Asynchronous on `stream`. */
 W8A8_API w8a8_status_t w8a8_debug_block_sums(const int8_t *xq, const int8_t *wq, int64_t M, int64_t K,
-                                    int64_t N, int32_t *out, void *stream);
+                                    int64_t N, int64_t m0, int64_t rows, int64_t n0, int64_t cols,
+                                    int32_t *out, void *stream);
 
 /* Synchronizes the current device and returns (and clears) the device error word:
  * W8A8_DEVERR_NONE or W8A8_DEVERR_TIMEOUT. */

@@ -137,6 +137,35 @@ def test_block_sums_config_slice(orc):
     np.testing.assert_array_equal(got.cpu().numpy(), orc.block_sums(xq, wq))
 
 
+@pytest.mark.parametrize("m0,rows,n0,cols", [(0, 384, 0, 640), (5, 100, 130, 300),
+                                              (129, 1, 639, 1), (256, 128, 256, 384)])
+def test_block_sums_windows(orc, m0, rows, n0, cols):
+    """Windows with any offsets and sizes: the main loop runs on the 128-aligned rows and
+    columns around them, and only the window is written."""
+    r = np.random.default_rng(m0 + rows + n0 + cols)
+    M, K, N = 384, 512, 640
+    xq = r.integers(-127, 128, (M, K)).astype(np.int8)
+    wq = r.integers(-127, 128, (N, K)).astype(np.int8)
+    got = w8.debug_block_sums(torch.from_numpy(xq).cuda(), torch.from_numpy(wq).cuda(),
+                              m0, rows, n0, cols)
+    np.testing.assert_array_equal(got.cpu().numpy(), orc.block_sums(xq, wq, m0, rows, n0, cols))
+
+
+def test_block_sums_mlp_up_full_size_windows(orc):
+    """The 16384 x 4096 x 16384 workload's own codes (quantized by the oracle): INT32 block
+    sums on three windows of the full-size GEMM (first tile, an unaligned window in the
+    middle, the last tile), bit for bit."""
+    wl = workload("mlp_up_16384")
+    lin = wl.linears[0]
+    xq, _ = orc.block_quantize(wl.x(16384, 4096))
+    wq, _ = orc.block_quantize(wl.w(lin))
+    dx, dw = torch.from_numpy(xq).cuda(), torch.from_numpy(wq).cuda()
+    for m0, rows, n0, cols in ((0, 128, 0, 256), (8191, 300, 9000, 333), (16256, 128, 16128, 256)):
+        got = w8.debug_block_sums(dx, dw, m0, rows, n0, cols)
+        np.testing.assert_array_equal(got.cpu().numpy(), orc.block_sums(xq, wq, m0, rows, n0, cols),
+                                      err_msg=f"window {m0},{rows},{n0},{cols}")
+
+
 # ------------------------------------------------------------------ W8A8 linear
 
 def _oracle_linear(orc, x, w, bias, m0=0, rows=None):
@@ -344,6 +373,12 @@ def test_error_codes():
         w8.linear(dev.float(), wt)
     with pytest.raises(ValueError):
         w8.linear(host, wt)
+    sums = torch.empty((100, 10, 2), dtype=torch.int32, device="cuda")
+    bs = L.w8a8_debug_block_sums
+    assert bs(q.data_ptr(), q.data_ptr(), 256, 256, 256, 200, 100, 0, 10, sums.data_ptr(), st) == 1
+    assert bs(q.data_ptr(), q.data_ptr(), 256, 256, 256, 0, 100, -1, 10, sums.data_ptr(), st) == 1
+    assert bs(q.data_ptr(), q.data_ptr(), 256, 200, 256, 0, 100, 0, 10, sums.data_ptr(), st) == 2
+    assert bs(q.data_ptr(), q.data_ptr(), 256, 256, 256, 0, 0, 0, 10, sums.data_ptr(), st) == 0
     torch.cuda.synchronize()
 
 
