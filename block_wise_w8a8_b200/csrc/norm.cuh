@@ -11,7 +11,13 @@
 // and y is block-quantized exactly as quant.cuh does (scale max|y| / 127, codes
 // rne(fl32(y / s)) clamped to +-127), without being written out.
 //
-// Work split.  A cluster of C = min(kMaxCluster, K / 128) CTAs (kMaxCluster = 4) owns one
+// Two forms.  rmsnorm_quantize_kernel below does all of it in one grid, each row's sum of
+// squares split across a cluster; row_rstd_kernel (end of this file) computes rstd alone,
+// one sequential FP64 chain per row, for quant::quantize_blocks_kernel<kRms / kRmsMod>
+// to normalise on load.  The library takes the second form from 192 rows per SM on, where
+// the row chains keep HBM busy (at M = 32768, K = 4096: 122 against 146 us).
+//
+// Work split of the one-grid form.  A cluster of C = min(kMaxCluster, K / 128) CTAs (kMaxCluster = 4) owns one
 // 128-row strip at a time; CTA r handles the strip's 128-column blocks kb = r, r + C, ...
 // (nb of them).  Each CTA streams its
 // blocks into a ring of six 32 KB shared-memory slots with 2-D TMA loads (two 64-column
@@ -503,6 +509,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     cluster_barrier();      // no CTA leaves while a peer may still send to it
+}
+
+// ------------------------------------------------------------------ row statistics ----
+// rstd of every row, with the sum of squares taken in FP64 in column order k = 0, 1, ...,
+// K - 1: one sequential chain per row, so every partial sum is rounded exactly as the
+// definition's running sum is, and rstd equals it bit for bit.  Each value is converted
+// exactly (BF16 -> FP32 by a shift, FP32 -> FP64 by the conversion instruction, which keeps
+// zeros, subnormals, infinities and NaNs) and its square is exact in FP64, so the fused
+// multiply-add rounds once, as the definition's separate square and add do.
+//
+// One thread per row.  A CTA of kSWarps consumer warps owns kSRows consecutive rows and
+// streams them in [kSRows x 64] boxes (2-D TMA, 128-byte swizzle, no multicast) through a
+// ring of kSStages slots, filled by one producer thread.  Thread r reads its row's eight
+// 16-byte chunks of a box in column order (chunk c sits at position c ^ (r % 8) of the
+// row's 128 bytes, so a warp's reads take the minimum four shared-memory wavefronts).
+//
+// The chain of K dependent FP64 operations per row sets a floor of roughly K times the
+// FP64 latency, whatever M is; with enough rows per SM (M of about 200 rows per SM and
+// up) the grid is bound by HBM instead.
+constexpr int kSWarps = 2;
+constexpr int kSRows = 32 * kSWarps;               // rows per CTA
+constexpr int kSStages = 6;
+constexpr int kSThreads = (kSWarps + 1) * 32;     // + the TMA producer warp
+constexpr uint32_t kSBoxBytes = kSRows * 128;      // [kSRows][64] BF16
+
+struct alignas(1024) SSmem {
+    uint16_t box[kSStages][kSRows * 64];
+    uint64_t full[kSStages];
+    uint64_t empty[kSStages];
+    int abort;
+};
+constexpr size_t kSSmemBytes = sizeof(SSmem) + 1024;
+static_assert(kSBoxBytes % 1024 == 0, "128-byte-swizzled boxes start on 1024-byte boundaries");
+
+// acc + the squares of eight BF16 values (four packed words, element 2i in the low half of
+// w[i]), added one at a time in element order.
+__device__ __forceinline__ double sumsq8(const uint4 v, double acc)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const double lo = static_cast<double>(bf16_lo(w[i]));
+        const double hi = static_cast<double>(bf16_hi(w[i]));
+        acc = fma(lo, lo, acc);
+        acc = fma(hi, hi, acc);
+    }
+    return acc;
+}
+
+__global__ void __launch_bounds__(kSThreads)
+    row_rstd_kernel(const __grid_constant__ CUtensorMap tmX, int64_t K, float eps,
+                    float *__restrict__ rstd)
+{
+    extern __shared__ uint8_t smem_raw[];
+    SSmem &sm = *reinterpret_cast<SSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    volatile int *abort = &sm.abort;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kSStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], kSWarps);
+        }
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // the quantizer that reads rstd may launch now; it waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int nbox = static_cast<int>(K / 64);
+    const int32_t row0 = static_cast<int32_t>(blockIdx.x) * kSRows;
+
+    if (warp == kSWarps) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmX);
+            uint32_t st = 0, ph = 0;
+            int b = 0;
+            for (; b < nbox; ++b) {
+                if (!mbar_wait(&sm.empty[st], ph ^ 1, abort))
+                    break;
+                mbar_arrive_expect_tx(&sm.full[st], kSBoxBytes);
+                tma_load_2d(sm.box[st], &tmX, &sm.full[st], b * 64, row0);
+                if (++st == kSStages) {
+                    st = 0;
+                    ph ^= 1;
+                }
+            }
+            if (b < nbox) {
+                // the copies already in flight land before shared memory is released
+                volatile int no_abort = 0;
+                for (int j = b > kSStages ? b - kSStages : 0; j < b; ++j)
+                    mbar_wait(&sm.full[j % kSStages], (j / kSStages) & 1, &no_abort, 100000000ull);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int r = threadIdx.x;                         // row within the CTA
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    double acc = 0.0;
+    uint32_t st = 0, ph = 0;
+    bool ok = true;
+    for (int b = 0; b < nbox; ++b) {
+        ok = mbar_wait(&sm.full[st], ph, abort);
+        if (__any_sync(0xFFFFFFFFu, !ok)) {
+            ok = false;
+            break;
+        }
+        const uint16_t *row = sm.box[st] + r * 64;
+#pragma unroll
+        for (uint32_t c = 0; c < 8; ++c)
+            acc = sumsq8(ld_shared_v4(row + ((c ^ sw) << 3)), acc);
+        // the sums depend on every value read: the slot is free again
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.empty[st]);
+        if (++st == kSStages) {
+            st = 0;
+            ph ^= 1;
+        }
+    }
+    if (ok)
+        rstd[row0 + r] = static_cast<float>(1.0 / sqrt(acc / static_cast<double>(K) + static_cast<double>(eps)));
 }
 
 } // namespace norm

@@ -177,9 +177,35 @@ static_assert((2 * kQStages) % kQGroups == 0,
               "item it - 2 S of the ring must belong to the same group as item it");
 
 
+// What is quantized: x itself, or x normalised on the way in (RMSNorm with the rstd a
+// previous grid computed, optionally followed by the scale-shift modulation; the
+// arithmetic of each is spelt out in norm.cuh).
+enum NormKind : int { kNone = 0, kRms = 1, kRmsMod = 2 };
+
+struct NormArgs {
+    const float *rstd;        // [rows], written by the grid this one depends on
+    const uint16_t *gamma;    // [K] BF16, or null (no affine factor)
+    const uint16_t *scale;    // [rows / T, K] BF16 (kRmsMod)
+    const uint16_t *shift;    // [rows / T, K] BF16 (kRmsMod)
+    int64_t T;                // rows sharing one modulation row; a multiple of 128
+};
+
+// Eight BF16 values (one 16-byte load) as FP32 numbers.
+__device__ __forceinline__ void unpack8_f32(uint4 v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16_lo(w[i]);
+        f[2 * i + 1] = bf16_hi(w[i]);
+    }
+}
+
+template <int kNorm>
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_blocks_kernel(const __grid_constant__ CUtensorMap tmX, int64_t K, int64_t nblocks,
-                           int64_t KB, int8_t *__restrict__ q, float *__restrict__ s)
+                           int64_t KB, int8_t *__restrict__ q, float *__restrict__ s,
+                           const NormArgs na)
 {
     extern __shared__ uint8_t smem_raw[];
     QSmem &sm = *reinterpret_cast<QSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -240,11 +266,37 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int row0 = gt >> 4;
     const int col = (gt & 15) * 8;
     constexpr int kRowStep = kQGroupWarps * 32 / 16;     // rows between a thread's chunks
+    // rstd comes from the grid this one was launched after: wait for its completion
+    if (kNorm != kNone)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t gi = 0;                                     // this group's block count
     for (int64_t blk = blockIdx.x + static_cast<int64_t>(g) * gridDim.x; blk < nblocks;
          blk += static_cast<int64_t>(kQGroups) * gridDim.x, ++gi) {
         const uint32_t it = gi * kQGroups + g;           // position in the ring's sequence
         const uint32_t st = it % kQStages, ph = (it / kQStages) & 1;
+        // the per-row and per-column factors of the normalisation, loaded before the block
+        float rs[kNorm != kNone ? kQChunks : 1], gm[8], am[8], sh[8];
+        if (kNorm != kNone) {
+            const int64_t mb = blk / KB, kb = blk - mb * KB;
+#pragma unroll
+            for (int j = 0; j < kQChunks; ++j)
+                rs[j] = __ldg(na.rstd + mb * 128 + row0 + kRowStep * j);
+            if (na.gamma != nullptr) {
+                unpack8_f32(__ldg(reinterpret_cast<const uint4 *>(na.gamma + kb * 128 + col)), gm);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    gm[e] = 1.0f;
+            }
+            if (kNorm == kRmsMod) {
+                const int64_t bm = (mb * 128) / na.T;
+                unpack8_f32(__ldg(reinterpret_cast<const uint4 *>(na.scale + bm * K + kb * 128 + col)), am);
+                unpack8_f32(__ldg(reinterpret_cast<const uint4 *>(na.shift + bm * K + kb * 128 + col)), sh);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    am[e] = __fadd_rn(1.0f, am[e]);
+            }
+        }
         // Slot st carries items it - S, it, it + S, ... of different groups.  A parity
         // wait cannot tell phase p from p + 2, so first make sure item it - S has been
         // consumed (the slot's full barrier is then in item it's phase or just past it).
@@ -253,14 +305,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
             break;
         if (!mbar_wait(&sm.full[st], ph, abort))
             break;
-        const uint16_t *tile = sm.tile[st];
+        uint16_t *tile = sm.tile[st];
         // pass 1 over the tile: absmax (the tile is read again for the codes, which keeps
-        // the registers free while the group waits for the block's scale)
+        // the registers free while the group waits for the block's scale).  When
+        // normalising, the BF16 values y are written back in place first.
         uint32_t m2 = 0;
 #pragma unroll
         for (int j = 0; j < kQChunks; ++j) {
-            const uint4 v = ld_shared_v4(tile + (row0 + kRowStep * j) * 128 + col);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint16_t *chunk = tile + (row0 + kRowStep * j) * 128 + col;
+            const uint4 v = ld_shared_v4(chunk);
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (kNorm != kNone) {
+                const float2 r2 = make_float2(rs[j], rs[j]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float2 n = __fmul2_rn(make_float2(bf16_lo(w[k]), bf16_hi(w[k])), r2);
+                    n = __fmul2_rn(n, make_float2(gm[2 * k], gm[2 * k + 1]));
+                    if (kNorm == kRmsMod) {
+                        // the shift is added with the scalar __fadd_rn, which is never
+                        // contracted with the product into a fused multiply-add; the
+                        // definition rounds the product and the sum separately
+                        n = __fmul2_rn(n, make_float2(am[2 * k], am[2 * k + 1]));
+                        n.x = __fadd_rn(n.x, sh[2 * k]);
+                        n.y = __fadd_rn(n.y, sh[2 * k + 1]);
+                    }
+                    w[k] = pack_bf16x2(n.x, n.y);
+                }
+                st_shared_v4(chunk, make_uint4(w[0], w[1], w[2], w[3]));
+            }
             m2 = absmax8_bits(w, m2);
         }
         uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
@@ -314,6 +386,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     static_cast<int8_t>(code_exact(v, sc));
             }
         }
+        // the normalised values this thread wrote into the slot are ordered before the
+        // next TMA fill of it (a write of the async proxy)
+        if (kNorm != kNone)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         // every lane is done with the slot (its loads were consumed above)
         __syncwarp();
         if (lane == 0)

@@ -28,7 +28,8 @@ struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     bool gemm_attr_set[5] = {false, false, false, false, false};
-    bool quant_attr_set = false;
+    bool quant_attr_set[3] = {false, false, false};    // by quant::NormKind
+    bool rstd_attr_set = false;
     bool norm_attr_set[4] = {false, false, false, false};
     int norm_max_clusters[norm::kMaxCluster + 1] = {};    // by cluster size, 0 = unknown
 };
@@ -223,31 +224,47 @@ w8a8_status_t launch_gemm(const void *a, const void *b, const gemm::Params &p0,
 
 // Block quantization of x [rows, cols] (both multiples of 128, buffers already checked):
 // one persistent CTA per SM, blocks streamed in by TMA.
-w8a8_status_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
-                              cudaStream_t stream)
+template <int kNorm>
+w8a8_status_t launch_quantize_t(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
+                                const quant::NormArgs &na, bool pdl, cudaStream_t stream)
 {
     int dev;
     W8A8_TRY(current_device(dev));
     CUtensorMap tm;
     W8A8_TRY(make_map(tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE));
+    auto kern = quant::quantize_blocks_kernel<kNorm>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_dev[dev].quant_attr_set) {
-            const cudaError_t e = cudaFuncSetAttribute(quant::quantize_blocks_kernel,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (!g_dev[dev].quant_attr_set[kNorm]) {
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        static_cast<int>(quant::kQSmemBytes));
             if (e != cudaSuccess)
                 return cuda_fail(e);
-            g_dev[dev].quant_attr_set = true;
+            g_dev[dev].quant_attr_set[kNorm] = true;
         }
     }
     const int64_t KB = cols / 128;
     const int64_t nblocks = (rows / 128) * KB;
     const int64_t grid = std::min<int64_t>(nblocks, g_dev[dev].sms);
-    quant::quantize_blocks_kernel<<<static_cast<unsigned>(grid), quant::kQThreads,
-                                    quant::kQSmemBytes, stream>>>(tm, cols, nblocks, KB, q, s);
-    return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(quant::kQThreads);
+    cfg.dynamicSmemBytes = quant::kQSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tm, cols, nblocks, KB, q, s, na);
+    return e == cudaSuccess ? launch_status() : cuda_fail(e);
+}
+
+w8a8_status_t launch_quantize(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
+                              cudaStream_t stream)
+{
+    return launch_quantize_t<quant::kNone>(x, rows, cols, q, s, quant::NormArgs{}, false, stream);
 }
 
 w8a8_status_t quantize_impl(const uint16_t *x, int64_t rows, int64_t cols, int8_t *q, float *s,
@@ -371,11 +388,37 @@ w8a8_status_t noalloc_scratch(int dev, void *&ptr)
     return W8A8_OK;
 }
 
-// Fused RMSNorm (+ modulation) + block quantization: clusters of C = min(4, K / 128) CTAs
-// (4 = norm::kMaxCluster), one cluster per 128-row strip at a time, as many clusters as
-// fit on the device.
+// rstd of every row of x [M, K] (M a multiple of norm::kSRows, K of 128): one CTA per
+// norm::kSRows rows.
+w8a8_status_t launch_row_rstd(const uint16_t *x, int64_t M, int64_t K, float eps, float *rstd,
+                              cudaStream_t stream)
+{
+    int dev;
+    W8A8_TRY(current_device(dev));
+    CUtensorMap tm;
+    W8A8_TRY(make_map(tm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, norm::kSRows, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+    auto kern = norm::row_rstd_kernel;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].rstd_attr_set) {
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       static_cast<int>(norm::kSSmemBytes));
+            if (e != cudaSuccess)
+                return cuda_fail(e);
+            g_dev[dev].rstd_attr_set = true;
+        }
+    }
+    kern<<<static_cast<unsigned>(M / norm::kSRows), norm::kSThreads, norm::kSSmemBytes, stream>>>(
+        tm, K, eps, rstd);
+    return launch_status();
+}
+
+// Fused RMSNorm (+ modulation) + block quantization in one grid: clusters of
+// C = min(4, K / 128) CTAs (4 = norm::kMaxCluster), one cluster per 128-row strip at a
+// time, as many clusters as fit on the device.
 template <bool kMod, bool kExactSq>
-w8a8_status_t launch_norm(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
+w8a8_status_t launch_norm_fused(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
 {
     int dev;
     W8A8_TRY(current_device(dev));
@@ -423,6 +466,57 @@ w8a8_status_t launch_norm(const uint16_t *x, const norm::Params &p, cudaStream_t
     if (e != cudaSuccess)
         return cuda_fail(e);
     return launch_status();
+}
+
+// RMSNorm (+ modulation) + block quantization as two grids: the rows' rstd
+// (norm::row_rstd_kernel), then the block quantizer normalising each block as it arrives
+// (quant::quantize_blocks_kernel<kRms / kRmsMod>), launched as a programmatic dependent
+// so that its set-up and first loads overlap the end of the first grid.  Without a
+// caller's rstd buffer the M floats come from the stream-ordered allocator.
+template <bool kMod>
+w8a8_status_t launch_norm_split(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
+{
+    const int64_t M = p.MB * 128;
+    float *rstd = p.rstd_out;
+    if (rstd == nullptr) {
+        void *tmp = nullptr;
+        const cudaError_t e = cudaMallocAsync(&tmp, static_cast<size_t>(M) * sizeof(float), stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        rstd = static_cast<float *>(tmp);
+    }
+    w8a8_status_t st = launch_row_rstd(x, M, p.K, p.eps, rstd, stream);
+    if (st == W8A8_OK) {
+        quant::NormArgs na;
+        na.rstd = rstd;
+        na.gamma = p.gamma;
+        na.scale = p.scale;
+        na.shift = p.shift;
+        na.T = p.T;
+        st = launch_quantize_t<kMod ? quant::kRmsMod : quant::kRms>(x, M, p.K, p.q, p.s, na, true, stream);
+    }
+    if (p.rstd_out == nullptr) {
+        const cudaError_t e = cudaFreeAsync(rstd, stream);
+        if (e != cudaSuccess && st == W8A8_OK)
+            st = cuda_fail(e);
+    }
+    return st;
+}
+
+// Rows per SM from which the two-grid form runs: its row-statistics grid is then bound by
+// HBM rather than by each row's chain of K dependent FP64 operations, and x read twice
+// costs less than the one-grid form's slot-bound pipeline (measured at K = 2048..16384).
+constexpr int64_t kNormSplitRowsPerSm = 192;
+
+template <bool kMod>
+w8a8_status_t launch_norm(const uint16_t *x, const norm::Params &p, cudaStream_t stream)
+{
+    int dev;
+    W8A8_TRY(current_device(dev));
+    if (p.MB * 128 >= kNormSplitRowsPerSm * g_dev[dev].sms)
+        return launch_norm_split<kMod>(x, p, stream);
+    return p.eps == 0.0f ? launch_norm_fused<kMod, true>(x, p, stream)
+                         : launch_norm_fused<kMod, false>(x, p, stream);
 }
 
 // Checks shared by both RMSNorm entry points; fills p (except the modulation fields).
@@ -542,7 +636,7 @@ w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t 
     if (M == 0)
         return W8A8_OK;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return eps == 0.0f ? launch_norm<false, true>(x, p, st) : launch_norm<false, false>(x, p, st);
+    return launch_norm<false>(x, p, st);
 }
 
 w8a8_status_t w8a8_rmsnorm_mod_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
@@ -566,7 +660,7 @@ w8a8_status_t w8a8_rmsnorm_mod_quantize_act(const w8a8_bf16_t *x, const w8a8_bf1
     p.shift = shift;
     p.T = T;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return eps == 0.0f ? launch_norm<true, true>(x, p, st) : launch_norm<true, false>(x, p, st);
+    return launch_norm<true>(x, p, st);
 }
 
 size_t w8a8_linear_workspace_bytes(int64_t M, int64_t K, int64_t N)

@@ -115,8 +115,18 @@ W8A8_API w8a8_status_t w8a8_quantize_act(const w8a8_bf16_t *x, int64_t M, int64_
  *   xs [M/128, K/128] FP32, and rstd_out [M] FP32 when not NULL.
  *   M, K multiples of 128 (else W8A8_ERR_SHAPE; M == 0 is a no-op), eps >= 0 and finite
  *   (else W8A8_ERR_INVALID_ARG); x, gamma, xq 16-byte aligned, xs and rstd_out 4-byte
- *   aligned.  Each block of x is loaded twice, once for the row sums and once for the
- *   codes; the second load is mostly served by L2. */
+ *   aligned.  Two forms, chosen by shape:
+ *   - M below 192 rows per SM: one grid; each row's sum of squares is split across a
+ *     cluster of CTAs, so its FP64 summation order differs from the running sum above,
+ *     and rstd may differ from it by one FP32 ulp on rows whose FP64 value lies within
+ *     about 1e-15 of an FP32 rounding boundary.  Each block of x is loaded twice, the
+ *     second time mostly from L2.
+ *   - M from 192 rows per SM on: a grid that sums each row's squares in column order (so
+ *     rstd equals the running-sum definition bit for bit), then the block quantizer
+ *     normalising each block as it arrives; x is read twice from HBM.  Without rstd_out
+ *     the M floats between the two grids come from the device's stream-ordered
+ *     allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *   Either way the codes and scales are those of y computed from the rstd returned. */
 W8A8_API w8a8_status_t w8a8_rmsnorm_quantize_act(const w8a8_bf16_t *x, const w8a8_bf16_t *gamma,
                                         float eps, int64_t M, int64_t K, int8_t *xq,
                                         float *xs, float *rstd_out, void *stream);

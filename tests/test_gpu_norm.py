@@ -1,14 +1,18 @@
-"""The fused RMSNorm + block quantizer, plain and modulated (TurboDiffusion article,
-inference list item 5; TurboT2VA paper, fused-operator paragraph), on the GPU through the
-C ABI, against the oracle.
+"""RMSNorm + block quantizer, plain and modulated (TurboDiffusion article, inference list
+item 5; TurboT2VA paper, fused-operator paragraph), on the GPU through the C ABI, against
+the oracle.
 
-rstd must equal the oracle's bit for bit except on rows where the two FP64 sums, taken in
-different orders, round to neighbouring FP32 values (at most one ulp, on a vanishing
-fraction of rows); given the kernel's rstd, codes and scales must equal the oracle's bit
-for bit.  Shapes cover every cluster size (C = min(4, K / 128)), 1 to 128 blocks per CTA
-and strip, block counts per CTA that are not a multiple of the four consumer groups or
-differ between the CTAs of a cluster, more strips than clusters, gamma absent, and eps = 0
-(the exact conversion path)."""
+The library runs one of two forms by shape: below 192 rows per SM a one-grid kernel whose
+row sums of squares are split across a cluster, from there on a row-statistics grid that
+sums each row in column order followed by the normalising block quantizer.  On the
+two-grid form rstd must equal the oracle's bit for bit on every row.  On the one-grid form
+it may differ on rows where the two FP64 sums, taken in different orders, round to
+neighbouring FP32 values (at most one ulp, on a vanishing fraction of rows).  Given the
+kernel's rstd, codes and scales must equal the oracle's bit for bit on both.  Shapes cover
+every cluster size (C = min(4, K / 128)), 1 to 128 blocks per CTA and strip, block counts
+per CTA that are not a multiple of the four consumer groups or differ between the CTAs of a
+cluster, more strips than clusters, gamma absent, and eps = 0 (the exact conversion path);
+the special rows (zeros, subnormals, eps = 0) and the near-tie sweep run on both forms."""
 import numpy as np
 import pytest
 import torch
@@ -38,14 +42,27 @@ def _rows(shape, seed, zero_row=True, tiny_row=True):
     return f64_to_bf16_bits(x)
 
 
-def _check(orc, x, g, eps, xq, xs, rstd, mod=None):
-    """mod = (scale_bits, shift_bits, T) for the modulated operation."""
+def split_rows():
+    """The smallest M (a multiple of 128) that takes the two-grid form on this GPU."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return -(-192 * sms // 128) * 128
+
+
+def _tile_rows(x, M):
+    """x repeated down to M rows (M a multiple of x's row count)."""
+    assert M % x.shape[0] == 0
+    return np.tile(x, (M // x.shape[0], 1))
+
+
+def _check(orc, x, g, eps, xq, xs, rstd, mod=None, exact_rstd=False):
+    """mod = (scale_bits, shift_bits, T) for the modulated operation; exact_rstd for
+    results of the two-grid form."""
     if mod is None:
         _, r_ref = orc.rmsnorm(x, g if g is not None else f64_to_bf16_bits(np.ones(x.shape[1])), eps)
     else:
         _, r_ref = orc.mod_rmsnorm(x, g, mod[0], mod[1], mod[2], eps)
     diff = np.nonzero(rstd.view(np.uint32) != r_ref.view(np.uint32))[0]
-    assert diff.size <= max(1, rstd.size // 100000), diff[:10]
+    assert diff.size <= (0 if exact_rstd else max(1, rstd.size // 100000)), diff[:10]
     for i in diff:
         assert abs(int(rstd.view(np.int32)[i]) - int(r_ref.view(np.int32)[i])) <= 1
     if mod is None:
@@ -96,25 +113,71 @@ def test_mod_rmsnorm_quantize(orc, M, K, T, with_gamma):
     _check(orc, x, g, 1e-6, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(), (sc, sh, T))
 
 
+@pytest.mark.parametrize("two_grid", [False, True])
 @pytest.mark.parametrize("modulated", [False, True])
-def test_eps_zero_exact_squares(orc, modulated):
+def test_eps_zero_exact_squares(orc, modulated, two_grid):
     """eps = 0 takes the exact FP64 conversion: rows of subnormal and mixed magnitudes."""
     M, K = 256, 1024
     x = _rows((M, K), 99, zero_row=False)
     # row 1 is subnormal but for one normal value, so that rstd stays finite
     x[1, 5] = f64_to_bf16_bits(np.array([1.0]))[0]
     x[3, 0] = f64_to_bf16_bits(np.array([2.0 ** -126]))[0]
+    if two_grid:
+        M = split_rows()
+        x = _tile_rows(x, M) if M % 256 == 0 else _tile_rows(x[:128], M)
     g = f64_to_bf16_bits(np.random.default_rng(5).uniform(0.5, 1.5, K))
     if modulated:
         r = np.random.default_rng(6)
-        sc = f64_to_bf16_bits(r.standard_normal((2, K)) * 0.5)
-        sh = f64_to_bf16_bits(r.standard_normal((2, K)) * 0.5)
+        sc = f64_to_bf16_bits(r.standard_normal((M // 128, K)) * 0.5)
+        sh = f64_to_bf16_bits(r.standard_normal((M // 128, K)) * 0.5)
         xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), dev_bf16(g), dev_bf16(sc),
                                                    dev_bf16(sh), 0.0)
-        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(), (sc, sh, 128))
+        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(), (sc, sh, 128),
+               exact_rstd=two_grid)
     else:
         xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), dev_bf16(g), 0.0)
-        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy())
+        _check(orc, x, g, 0.0, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(),
+               exact_rstd=two_grid)
+
+
+@pytest.mark.parametrize("K", [128, 640, 4096])
+@pytest.mark.parametrize("modulated", [False, True])
+@pytest.mark.parametrize("with_gamma", [True, False])
+def test_two_grid_form(orc, K, modulated, with_gamma):
+    """The two-grid form on every row: rows of widely spread magnitudes, a zero row, a
+    subnormal row and zeros inside rows (_rows), rstd bit-exact on every row; one
+    modulation row per 256 rows; then the same call without a caller's rstd buffer gives
+    the same codes and scales."""
+    M = split_rows()
+    x = _rows((M, K), K + 3)
+    r = np.random.default_rng(K)
+    g = f64_to_bf16_bits(r.uniform(0.5, 1.5, K)) if with_gamma else None
+    gd = None if g is None else dev_bf16(g)
+    T = 256 if M % 256 == 0 else 128
+    sc = f64_to_bf16_bits(r.standard_normal((M // T, K)) * 0.5)
+    sh = f64_to_bf16_bits(r.standard_normal((M // T, K)) * 0.5)
+    scd, shd = dev_bf16(sc), dev_bf16(sh)
+    if modulated:
+        xq, xs, rstd = w8.rmsnorm_mod_quantize_act(dev_bf16(x), gd, scd, shd, 1e-6)
+    else:
+        xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), gd, 1e-6)
+    _check(orc, x, g, 1e-6, xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy(),
+           (sc, sh, T) if modulated else None, exact_rstd=True)
+    # without rstd_out: the library takes M floats of stream-ordered scratch
+    L = w8.lib()
+    st = w8._stream(torch.device("cuda"))
+    xd = dev_bf16(x)
+    q2 = torch.empty_like(xq)
+    s2 = torch.empty_like(xs)
+    P = lambda t: None if t is None else t.data_ptr()
+    if modulated:
+        rc = L.w8a8_rmsnorm_mod_quantize_act(P(xd), P(gd), P(scd), P(shd), T, 1e-6,
+                                             M, K, P(q2), P(s2), None, st)
+    else:
+        rc = L.w8a8_rmsnorm_quantize_act(P(xd), P(gd), 1e-6, M, K, P(q2), P(s2), None, st)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.equal(q2, xq) and torch.equal(s2.view(torch.int32), xs.view(torch.int32))
 
 
 @pytest.mark.parametrize("modulated", [False, True])
@@ -133,13 +196,19 @@ def test_hires_chain_norm_sampled(orc, modulated):
     else:
         xq, xs, rstd = w8.rmsnorm_quantize_act(dev_bf16(x), dev_bf16(g), eps)
     xq, xs, rstd = xq.cpu().numpy(), xs.cpu().numpy(), rstd.cpu().numpy()
+    exact = M >= split_rows()
+    if exact:
+        # every row's rstd (the oracle's normalisation of all rows is cheap; its
+        # quantization of all of them is not needed for this)
+        _, r_ref = orc.rmsnorm(x, g, eps)
+        np.testing.assert_array_equal(rstd.view(np.uint32), r_ref.view(np.uint32))
     for mb in (0, 137, 255):
         rows = slice(mb * 128, (mb + 1) * 128)
         xr = x[rows]
         if modulated:
-            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows], (sc, sh, 128))
+            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows], (sc, sh, 128), exact_rstd=exact)
         else:
-            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows])
+            _check(orc, xr, g, eps, xq[rows], xs[mb:mb + 1], rstd[rows], exact_rstd=exact)
 
 
 def test_mod_errors():
@@ -163,17 +232,23 @@ def test_mod_errors():
     torch.cuda.synchronize()
 
 
+@pytest.mark.parametrize("two_grid", [False, True])
 @pytest.mark.parametrize("modulated", [False, True])
 @pytest.mark.parametrize("eps", [0.0, 1e-6])
-def test_fused_codes_near_ties_exhaustive(orc, modulated, eps):
+def test_fused_codes_near_ties_exhaustive(orc, modulated, eps, two_grid):
     """Every BF16 value of both signs in [A/512, A] as a normalised value, for five block
     absmaxes A that are not powers of two: the rows' RMS is 1 (rstd exactly 1.0), so the
-    fused kernel quantizes the input values themselves, and its codes and scales must
-    equal the oracle's bit for bit, near-ties included (eps = 0 takes the exact-square
-    instantiation, eps = 1e-6 the scaled one; modulated with zero scale and shift)."""
+    kernel quantizes the input values themselves, and its codes and scales must equal the
+    oracle's bit for bit, near-ties included (one-grid form: eps = 0 takes the exact-square
+    instantiation, eps = 1e-6 the scaled one; modulated with zero scale and shift).  On
+    the two-grid form the sweep's strips are repeated down to the form's row count."""
     from norm_sweep import ABSMAXES, unit_rms_rows
     K = 4096
     x = unit_rms_rows(K, eps)
+    if two_grid:
+        base = x.shape[0]
+        M = -(-split_rows() // base) * base
+        x = _tile_rows(x, M)
     M = x.shape[0]
     if modulated:
         z = np.zeros((1, K), dtype=np.uint16)
