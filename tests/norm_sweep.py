@@ -1,4 +1,5 @@
-"""Inputs for the exhaustive near-tie sweep through the fused RMSNorm's code arithmetic.
+"""Inputs for the exhaustive near-tie sweep through the RMSNorm + quantizer's code arithmetic
+(both of the library's forms).
 
 Every row's sum of squares is built so that its RMS is 1 to far better than FP32
 precision (Sum x^2 = K (1 - eps) up to a remainder below 2^-40 of it), so rstd is exactly
