@@ -17,13 +17,14 @@
 // to normalise on load.  The library takes the second form from 192 rows per SM on, where
 // the row chains keep HBM busy (at M = 32768, K = 4096: 122 against 146 us).
 //
-// Work split of the one-grid form.  A cluster of C = min(kMaxCluster, K / 128) CTAs (kMaxCluster = 4) owns one
-// 128-row strip at a time; CTA r handles the strip's 128-column blocks kb = r, r + C, ...
-// (nb of them).  Each CTA streams its
-// blocks into a ring of six 32 KB shared-memory slots with 2-D TMA loads (two 64-column
-// boxes per block, 128-byte swizzle, no multicast), each block twice: once for the sums of
-// squares and once for the codes.  The second load comes about one strip later and is
-// served by L2 (a cluster has about two 1 MB strips in flight), so x crosses HBM once.
+// Work split of the one-grid form.  A cluster of C = min(kMaxCluster, K / 128) CTAs
+// (kMaxCluster = 4) owns one 128-row strip at a time; CTA r handles the strip's 128-column
+// blocks kb = r, r + C, ... (nb of them).  Each CTA streams its blocks into a ring of six
+// 32 KB shared-memory slots with 2-D TMA loads (two 64-column boxes per block, 128-byte
+// swizzle, no multicast), each block twice: once for the sums of squares and once for the
+// codes.  The second load comes about one strip later and is meant to be served by L2 (a
+// cluster has about two 1 MB strips in flight); at 32768 x 4096 about two thirds of those
+// loads miss it.
 //
 //   pass 1   each thread owns one row of a block and sums its squares in FP64.  The FP64
 //            operand is built from the BF16 bits with two integer operations, as |x| *
