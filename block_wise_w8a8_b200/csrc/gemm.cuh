@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int c = 0; c < 8; ++c) {
                             uint32_t r[16];
                             tmem_ld16(tb + c * 16, r);
-                            tmem_wait_ld();
+                            tmem_wait_ld(r);
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 float2 v = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int c = 0; c < 4; ++c) {
                         uint32_t r[32];
                         tmem_ld32(tb + c * 32, r);
-                        tmem_wait_ld();
+                        tmem_wait_ld(r);
                         const int64_t wm = m - p.dm0;
                         if (n0 < p.N && wm >= 0 && wm < p.drows) {
 #pragma unroll
@@ -691,7 +691,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tb + c * 32, r);
-                    tmem_wait_ld();
+                    tmem_wait_ld(r);
                     const int64_t nc = n0 + c * 32;
                     if (nc < p.N) {
                         uint16_t *dst = p.y + m * p.N + nc;
@@ -750,7 +750,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tb + c * 32, r);
-                    tmem_wait_ld();
+                    tmem_wait_ld(r);
                     const int64_t nc = n0 + c * 32;
                     if (m < p.M && nc < p.N) {
                         uint16_t *dst = p.y + m * p.N + nc;
