@@ -223,7 +223,10 @@ def rowwise_linear(x, wq, ws, bias=None, out=None):
 
 def rmsnorm_quantize_act(x, gamma, eps=1e-6, xq=None, xs=None, rstd=None):
     """RMSNorm (FP64 row sums, FP32 rstd, bf16((x * rstd) * gamma); gamma may be None)
-    fused with the block quantizer -> (xq, xs, rstd)."""
+    fused with the block quantizer (the normalised values are never stored) -> (xq, xs,
+    rstd).  From 192 rows per SM the row sums follow the definition's column order, so rstd
+    is exactly the definition's; below that a one-grid kernel splits each row over a
+    cluster and rstd may differ by one FP32 ulp on rare rows (see include/w8a8.h)."""
     _need(x, torch.bfloat16, "x")
     if gamma is not None:
         _need(gamma, torch.bfloat16, "gamma")
